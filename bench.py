@@ -45,6 +45,9 @@ def parse_args():
     p.add_argument("--group", type=int, default=None,
                    help="RHT group size (default: the workload's first group)")
     p.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    p.add_argument("--scaling", default="weak", choices=("weak", "strong"),
+                   help="weak: every rank runs its own batch of M tokens; strong: one batch of M "
+                        "tokens split over the ranks by rows (dp.run_sharded)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--record-traffic", metavar="NCU_CSV",
@@ -91,7 +94,8 @@ def l2_bytes(dev) -> int:
     return int(size) if size else 126 * 2**20
 
 
-KERNEL_SOURCES = ("capi.cu", "internal.h", "ptx.cuh", "rht_quant.cuh", "gemm_common.cuh",
+KERNEL_SOURCES = ("capi.cu", "internal.h", "ptx.cuh", "rht_quant.cuh", "rht_quant_ring.cuh",
+                  "gemm_common.cuh",
                   "w4a4_gemm.cuh", "w8a8_gemm.cuh", "nvfp4_gemm.cuh")
 
 
@@ -454,10 +458,18 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     from rotation_w4a4_quantized_b200 import binding as B
-    from rotation_w4a4_quantized_b200.dp import job_throughput, slowest_rank_ms
+    from rotation_w4a4_quantized_b200.dp import (job_throughput, local_rows, run_sharded,
+                                                 slowest_rank_ms)
 
-    X, W, _ = make_inputs(w, seed=w.seed + 1000 * rank if rank else None)
+    strong = args.scaling == "strong"
+    # weak: each rank its own batch of M tokens (its own seed); strong: one global batch, the
+    # same bytes on every rank, of which each rank takes its rows
+    X, W, _ = make_inputs(w, seed=None if strong or not rank else w.seed + 1000 * rank)
     dev = torch.device("cuda", local_rank)
+    Xg = X
+    if strong:
+        X = local_rows(Xg, rank, world).contiguous()
+    Ml = X.shape[0]                               # token rows this rank runs per step
     Xd, Wd = X.to(dev), W.to(dev)
     int8 = args.variant == "w8a8"
     mx = args.variant == "mxfp4"
@@ -468,7 +480,7 @@ def main():
         K_pad = B.nvfp4_k(w.K, g)                 # the FP4 paths run over K4 (multiple of 64)
         qw0, sfw0 = B.prepack_weight_mxfp4(Wd, g)
         ldq = B.packed_stride(K_pad)
-        sf_bytes = B.mxfp4_scale_bytes(w.M, w.K, g, False)
+        sf_bytes = B.mxfp4_scale_bytes(Ml, w.K, g, False)
 
         def quant(st):
             B.rotate_quant_act_mxfp4(st["X"], g, q=st["qx"], sf=st["sfx"])
@@ -482,7 +494,7 @@ def main():
         K_pad = B.nvfp4_k(w.K, g)                 # the NVFP4 path runs over K4 (multiple of 64)
         qw0, sfw0, gw0 = B.prepack_weight_nvfp4(Wd, g)
         ldq = B.packed_stride(K_pad)
-        sf_bytes = B.nvfp4_scale_bytes(w.M, w.K, g, False)
+        sf_bytes = B.nvfp4_scale_bytes(Ml, w.K, g, False)
 
         def quant(st):
             B.rotate_quant_act_nvfp4(st["X"], g, q=st["qx"], sf=st["sfx"], g=st["sx"])
@@ -513,10 +525,10 @@ def main():
             return layer_fn(X_, qw0, sw0, g, K_pad)
 
     def new_set():
-        st = {"X": Xd.clone(), "qx": torch.empty(w.M, ldq, dtype=u8, device=dev),
-              "Y": torch.empty(w.M, w.N, dtype=bf16, device=dev), "qw": qw0.clone()}
+        st = {"X": Xd.clone(), "qx": torch.empty(Ml, ldq, dtype=u8, device=dev),
+              "Y": torch.empty(Ml, w.N, dtype=bf16, device=dev), "qw": qw0.clone()}
         if not mx:                                # MXFP4 has no per-row scale
-            st["sx"] = torch.empty(w.M, dtype=f32, device=dev)
+            st["sx"] = torch.empty(Ml, dtype=f32, device=dev)
         if fp4:
             st.update(sfw=sfw0.clone(), sfx=torch.empty(sf_bytes, dtype=u8, device=dev))
             if not mx:
@@ -539,6 +551,12 @@ def main():
         linear(sets[i % n_sets])
     torch.cuda.synchronize()
     assert B.device_status() == 0
+    if strong:
+        # the split-and-gather of one global batch reproduces the unsplit layer bit for bit
+        Xgd = Xg.to(dev)
+        y_split = run_sharded(Xgd, layer, rank, world)
+        assert torch.equal(y_split, layer(Xgd)), "row-split layer differs from the whole batch"
+        del Xgd, y_split
 
     K = args.steps
 
@@ -606,8 +624,15 @@ def main():
         t_wall1 = time.time()
     del q_sets
     ms_per_step = total_ms / K
-    ops = 2.0 * w.M * w.N * K_pad
-    value = job_throughput(ops, world, ms_per_step) / 1e12
+    ops = 2.0 * Ml * w.N * K_pad
+
+    def job_rate(ms):
+        """Whole-job ops/s: strong scaling divides the one global batch by the slowest rank."""
+        if strong:
+            return 2.0 * w.M * w.N * K_pad / (ms * 1e-3)
+        return job_throughput(ops, world, ms)
+
+    value = job_rate(ms_per_step) / 1e12
     clocks = clk.summary(t_wall0, t_wall1)
     assert B.device_status() == 0
 
@@ -616,15 +641,19 @@ def main():
     peak_ratio = 4.0 if fp4 else 2.0
     int8_peak = peak_ratio * bf16_tflops
     gemm_avg, quant_avg = gemm_ms, quant_ms
-    quant_bytes = w.M * w.K * 2 + w.M * (K_pad if int8 else K_pad // 2)
+    quant_bytes = Ml * w.K * 2 + Ml * (K_pad if int8 else K_pad // 2)
     if mx:
-        quant_bytes += w.M * K_pad // 32                  # one e8m0 scale per 32 K
+        quant_bytes += Ml * K_pad // 32                  # one e8m0 scale per 32 K
     elif fp4:
-        quant_bytes += w.M * K_pad // 16 + w.M * 4        # e4m3 per 16 K, fp32 row scale
+        quant_bytes += Ml * K_pad // 16 + Ml * 4        # e4m3 per 16 K, fp32 row scale
     else:
-        quant_bytes += w.M * 4                            # fp32 row scale
+        quant_bytes += Ml * 4                            # fp32 row scale
     quant_gbs = quant_bytes / (quant_avg / 1e3) / 1e9
     config = workload_desc(w, g, K_pad, args.variant)
+    config["parallelism"] = (f"dp{world}: one batch of {w.M} tokens split by rows ({Ml} on rank "
+                             f"0), replicated weights, no collective on the data path" if strong
+                             else f"dp{world}: {w.M} tokens per rank, replicated weights, no "
+                                  f"collective on the data path")
     config["l2"] = (f"inputs larger than L2: {n_sets} rotating copies of every operand "
                     f"({set_bytes / 1e6:.0f} MB each), no flush inside the timed region")
     del sets
@@ -639,7 +668,7 @@ def main():
     if not args.no_e2e:
         from rotation_w4a4_quantized_b200.pipeline import HostPipeline
         Xh = X.pin_memory()
-        Yhs = [torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        Yhs = [torch.empty(Ml, w.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         h2d_bytes = Xh.numel() * Xh.element_size()
         d2h_bytes = Yhs[0].numel() * Yhs[0].element_size()
         ke = max(1, min(K, 200))
@@ -663,11 +692,11 @@ def main():
         if world > 1:
             dist.barrier()
         s_ms = slowest_rank_ms(sum(a.elapsed_time(b) for a, b in eev)) / ke
-        e2e_serial = {"value": job_throughput(ops, world, s_ms) / 1e12, "unit": "TOPS",
+        e2e_serial = {"value": job_rate(s_ms) / 1e12, "unit": "TOPS",
                       "ms_per_step": s_ms, "steps": ke, "h2d_bytes_per_step": h2d_bytes,
                       "d2h_bytes_per_step": d2h_bytes}
 
-        pipe = HostPipeline(layer, w.M, w.K, device=dev, depth=2)
+        pipe = HostPipeline(layer, Ml, w.K, device=dev, depth=2)
         pipe.run([Xh] * 4, [Yhs[i % 2] for i in range(4)])       # warm-up
         torch.cuda.synchronize()
         if world > 1:
@@ -682,7 +711,7 @@ def main():
         if world > 1:
             dist.barrier()
         e_ms = slowest_rank_ms(p0.elapsed_time(p1)) / ke
-        e2e = {"value": job_throughput(ops, world, e_ms) / 1e12, "unit": "TOPS",
+        e2e = {"value": job_rate(e_ms) / 1e12, "unit": "TOPS",
                "ms_per_step": e_ms, "steps": ke, "h2d_bytes_per_step": h2d_bytes,
                "d2h_bytes_per_step": d2h_bytes,
                "how": "HostPipeline: per step, H2D of the activations from pinned host memory, "
@@ -694,10 +723,10 @@ def main():
     # rotating copies of its operands larger than L2, one event pair around the whole run
     bf16_us = None
     if rank == 0:
-        bsets = [(Xd.clone(), Wd.clone(), torch.empty(w.M, w.N, dtype=bf16, device=dev))]
+        bsets = [(Xd.clone(), Wd.clone(), torch.empty(Ml, w.N, dtype=bf16, device=dev))]
         b_bytes = sum(t.numel() * t.element_size() for t in bsets[0])
         nb = max(3, -(-3 * l2_bytes(dev) // b_bytes))
-        bsets += [(Xd.clone(), Wd.clone(), torch.empty(w.M, w.N, dtype=bf16, device=dev))
+        bsets += [(Xd.clone(), Wd.clone(), torch.empty(Ml, w.N, dtype=bf16, device=dev))
                   for _ in range(nb - 1)]
         for i in range(3 * nb):
             xb, wb, yb = bsets[i % nb]
@@ -744,7 +773,7 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "e2m1" if fp4 else "s8",
         "data": "synthetic",
@@ -782,7 +811,7 @@ def main():
         "int8_library_gemm": int8_lib,
         "bf16_linear": None if bf16_us is None else {
             "what": "unquantised bf16 X @ W^T (cuBLAS) of the same shape, reported baseline",
-            "us": bf16_us, "tflops": 2.0 * w.M * w.N * w.K / (bf16_us / 1e6) / 1e12,
+            "us": bf16_us, "tflops": 2.0 * Ml * w.N * w.K / (bf16_us / 1e6) / 1e12,
             "layer_speedup": bf16_us / (ms_per_step * 1e3)},
     }
     print(json.dumps(line), flush=True)

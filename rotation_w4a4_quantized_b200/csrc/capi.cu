@@ -11,6 +11,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 #include "rht_quant.cuh"
+#include "rht_quant_ring.cuh"
 #include "w4a4_gemm.cuh"
 #include "w8a8_gemm.cuh"
 #include "nvfp4_gemm.cuh"
@@ -24,7 +25,7 @@ bool valid_group(int g) { return g == 16 || g == 64 || g == 256 || g == 1024; }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Per device: whether it was queried, and whether it is sm_100 family.
+// Per device: whether it was queried, and whether it is an sm_100 part.
 int g_dev_ok[kMaxDevices] = {};
 bool g_dev_checked[kMaxDevices] = {};
 
@@ -35,12 +36,15 @@ int check_device() {
     return CONVROT_ERR_DEVICE;
   }
   if (dev < kMaxDevices && g_dev_checked[dev]) return g_dev_ok[dev] ? CONVROT_OK : CONVROT_ERR_DEVICE;
-  int major = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+  // the library is built for sm_100a alone: arch-specific code does not load on other
+  // compute capability 10.x parts
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
     cudaGetLastError();
     return CONVROT_ERR_DEVICE;
   }
-  const bool ok = (major == 10);
+  const bool ok = (major == 10 && minor == 0);
   if (dev < kMaxDevices) {
     g_dev_ok[dev] = ok ? 1 : 0;
     g_dev_checked[dev] = true;

@@ -39,8 +39,9 @@ struct TileGrid {
 // Dequantise one finished accumulator block -- this warp's 32 TMEM lanes (rows row0..row0+31)
 // x BN columns starting at n0 -- and store it:
 //   Y[m,n] = bf16_rne((float(acc >> kShift) * sx[m]) * sw[n] + float(bias[n]))
-// (kShift = 8 when the accumulator holds 256 * acc; the shift is folded into the row scale,
-// which is exact). As soon as the last columns are in registers the warp arrives on
+// (kShift = 8 when the accumulator holds 256 * acc: the arithmetic shift of the integer
+// accumulator is exact, so the formula runs on the exact acc whatever the row scale's
+// magnitude). As soon as the last columns are in registers the warp arrives on
 // `acc_empty_addr` (a shared::cluster barrier address) so the MMA can reuse the accumulator.
 // bf16 blocks of 32 x 32 are staged in shared memory with the 64-byte swizzle and written by
 // TMA stores when `tma_out`; otherwise element stores are used. kRawS32 stores acc >> kShift.
@@ -63,8 +64,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, int row0, int n
   const int lane = threadIdx.x & 31;
   const int m = row0 + lane;
   const bool row_ok = m < M;
-  constexpr float kUnit = 1.0f / static_cast<float>(1 << kShift);
-  const float sxm = !kScaled ? 1.f : ((row_ok && sx) ? sx[m] * kUnit : 0.f);
+  const float sxm = !kScaled ? 1.f : ((row_ok && sx) ? sx[m] : 0.f);
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += kEpiCols) {
     uint32_t acc[kEpiCols];
@@ -94,9 +94,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, int row0, int n
       uint32_t pkd[kEpiCols / 2];
 #pragma unroll
       for (int i = 0; i < kEpiCols; i += 2) {
-        const float a0 = kF32Acc ? __uint_as_float(acc[i]) : static_cast<float>(static_cast<int32_t>(acc[i]));
+        const float a0 = kF32Acc ? __uint_as_float(acc[i])
+                                 : static_cast<float>(static_cast<int32_t>(acc[i]) >> kShift);
         const float a1 = kF32Acc ? __uint_as_float(acc[i + 1])
-                                 : static_cast<float>(static_cast<int32_t>(acc[i + 1]));
+                                 : static_cast<float>(static_cast<int32_t>(acc[i + 1]) >> kShift);
         float v0 = a0 * sxm;
         float v1 = a1 * sxm;
         v0 = v0 * __shfl_sync(0xffffffffu, sw_l, i);

@@ -163,19 +163,22 @@ __host__ __device__ constexpr int log4_of() {
 
 // H_1024 on the 64 values this thread owns, in place (unnormalised: entries +-1). Digits 0..2
 // run in registers; then the 16 threads of a group exchange their values once through xbuf (one
-// 256-byte row per thread, 16-byte chunk index XOR (row & 7)) and run digits 3 and 4. On return
-// v[] holds the values in the layout documented at store_codes().
+// 256-byte row per thread, 16-byte chunk index XOR (row & 7)) and run digits 3 and 4. On entry
+// v[4 ch .. 4 ch + 3] holds the chunk's 4-column piece ch ^ perm (perm = 0: natural order; a
+// digit-wise permutation of the pieces leaves digits 0..2 unchanged); on return v[] holds the
+// values in the layout documented at store_codes().
 template <int G>
 __device__ __forceinline__ void transform_chunk(float (&v)[kChunk], float4* __restrict__ xbuf,
-                                                int tid) {
+                                                int tid, int perm = 0) {
   static_assert(G == 1024, "G <= 256 use the slot layout (transform_slots)");
   radix4_stage<1>(v);
   radix4_stage<4>(v);
   radix4_stage<16>(v);
   float4* mine = xbuf + tid * 16;
+  const int wx = perm ^ (tid & 7);
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch)
-    mine[ch ^ (tid & 7)] = make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+    mine[ch ^ wx] = make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
   __syncwarp();
   // group = 16 threads; thread j takes column chunk j (4 columns) of all 16 rows.
   const int j = tid & 15;
@@ -1156,9 +1159,20 @@ cudaError_t launch_reg_t(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, i
                            team_rows, fp4);
 }
 
+// The row-streaming kernel (rht_quant_ring.cuh); cudaErrorNotSupported when the shape does not
+// fit it.
+template <int G, int QM>
+cudaError_t launch_ring(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
+                        uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream);
+
 template <int G, int QM>
 cudaError_t launch_g(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
                      uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream) {
+  // K a multiple of 8 and rows of at most 16384 columns: whole rows stream into a shared ring
+  {
+    const cudaError_t e = launch_ring<G, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if constexpr (G == 1024) {
     // long groups: the TMA-staged kernel when the row fits its ring (K a multiple of 64)
     const cudaError_t e = (K_pad / kChunk <= 128)

@@ -29,6 +29,42 @@ def shard_rows(M: int, rank: int, world: int) -> Tuple[int, int]:
     return start, stop
 
 
+def local_rows(X, rank: int, world: int):
+    """This rank's rows of a batch (a view: no copy), as shard_rows assigns them."""
+    start, stop = shard_rows(X.shape[0], rank, world)
+    return X[start:stop]
+
+
+def gather_rows(y_local, M: int, rank: int, world: int, group=None):
+    """All ranks' output rows in global order (every rank receives the whole [M, ...] result).
+
+    Shards differ by at most one row; each is padded to the largest before the all-gather
+    (collectives move equal-sized buffers) and trimmed after it."""
+    import torch
+    import torch.distributed as dist
+
+    if world == 1:
+        return y_local
+    start, stop = shard_rows(M, rank, world)
+    if y_local.shape[0] != stop - start:
+        raise ValueError(f"rank {rank} holds {y_local.shape[0]} rows, expected {stop - start}")
+    rows = -(-M // world)
+    pad = torch.zeros((rows,) + tuple(y_local.shape[1:]), dtype=y_local.dtype,
+                      device=y_local.device)
+    pad[: y_local.shape[0]] = y_local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat([parts[r][: b - a] for r, (a, b) in
+                      enumerate(shard_rows(M, r, world) for r in range(world))])
+
+
+def run_sharded(X, layer, rank: int, world: int, gather: bool = True, group=None):
+    """One global batch split over the ranks by rows: `layer` runs on this rank's rows (no
+    communication on the data path); with `gather`, the outputs are all-gathered in row order."""
+    y = layer(local_rows(X, rank, world))
+    return gather_rows(y, X.shape[0], rank, world, group) if gather else y
+
+
 def slowest_rank_ms(local_ms: float, group=None) -> float:
     """Max over ranks of a per-rank device time (ms); the job is as fast as its slowest rank."""
     import torch

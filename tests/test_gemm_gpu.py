@@ -106,6 +106,35 @@ def test_dequant_epilogue_on_oracle_codes(cuda_lib, M, N, K_pad, with_bias):
     check_y_elementwise(bf16_to_f64(y), acc, sx, sw, b64, "dequant")
 
 
+def test_dequant_tiny_row_scales(cuda_lib):
+    """Row scales far below the fp32 normal range against weight scales far above it: the
+    epilogue multiplies the exact integer accumulator by the scale as stored ("comfy-kitchen PR
+    #65", the fp32 fix of int4_linear: the scales multiply the exact integer product). Row 3's
+    scale, 383 * 2^-149, is a subnormal fp32 whose product with any accumulator is exact; a
+    1/256 folded into it would round it to 2^-149 (33 % off). Row 4 is a bf16 activation row of
+    magnitude ~1e-36 (scale ~1.4e-37)."""
+    M, N, K_pad = 64, 96, 512
+    rng = np.random.default_rng(11)
+    px = random_packed(M, K_pad, seed=21)
+    pw = random_packed(N, K_pad, seed=22)
+    sx = rng.uniform(0.01, 3.0, M).astype(np.float32)
+    sx[3] = np.array([383], dtype=np.uint32).view(np.float32)[0]
+    sx[4] = np.float32(1e-36 / 7)
+    sw = rng.uniform(1e-4, 5e-3, N).astype(np.float32)
+    sw[N // 2:] = np.float32(2.0 ** 100)                       # large-magnitude weight rows
+    sw[N // 2:] /= np.float32(1.0) + (np.arange(N - N // 2, dtype=np.float32) % 7)
+    qx, qw = upload_packed(px, K_pad, cuda_lib), upload_packed(pw, K_pad, cuda_lib)
+    y = cuda_lib.w4a4_linear(qx, torch.from_numpy(sx).cuda(), qw, torch.from_numpy(sw).cuda(),
+                             K_pad)
+    acc = O.int_gemm(O.unpack_int4(px), O.unpack_int4(pw))
+    yg = bf16_to_f64(y)
+    check_y_elementwise(yg, acc, sx, sw, None, "tiny row scales")
+    big = slice(N // 2, N)
+    ref = O.dequant(acc, sx, sw)[3, big]
+    assert np.all(np.abs(yg[3, big] - ref) <= 2.0 ** -8 * np.abs(ref)), "row 3 off"
+    assert np.count_nonzero(ref) > 0
+
+
 def test_output_stride_and_zero_sizes(cuda_lib):
     K_pad, M, N = 256, 70, 136
     px, pw = random_packed(M, K_pad, 1), random_packed(N, K_pad, 2)

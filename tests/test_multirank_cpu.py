@@ -75,6 +75,66 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
+def _strong_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import convrot_oracle as O
+    from rotation_w4a4_quantized_b200.dp import run_sharded
+    from synthetic import CONFIGS, make_inputs
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        w = CONFIGS["tiny"]
+        X, W, bias = make_inputs(w, with_bias=True)
+        X = X[:61]                                  # a batch that does not split evenly
+        W64 = W.float().numpy().astype(np.float64)
+        b64 = bias.float().numpy().astype(np.float64)
+        seen = []
+
+        def layer(x_local):
+            # the CPU stand-in for the device layer: the oracle on this rank's rows
+            seen.append(x_local.shape[0])
+            res = O.w4a4_linear(x_local.float().numpy().astype(np.float64), W64, w.group,
+                                bias=b64)
+            return torch.from_numpy(res["y"])
+
+        y = run_sharded(X, layer, rank, world)
+        out.put((rank, seen[0], y.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_strong_split_and_gather():
+    """run_sharded (the split-and-gather bench.py's strong-scaling mode calls): each rank's
+    layer sees only its rows, and every rank ends with the unsharded output."""
+    from oracle import convrot_oracle as O
+    from synthetic import CONFIGS, make_inputs
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_strong_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict((r, (n, y)) for r, n, y in (q.get(timeout=120) for _ in range(2)))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    w = CONFIGS["tiny"]
+    X, W, bias = make_inputs(w, with_bias=True)
+    ref = O.w4a4_linear(X[:61].float().numpy().astype(np.float64),
+                        W.float().numpy().astype(np.float64), w.group,
+                        bias=bias.float().numpy().astype(np.float64))["y"]
+    assert [got[r][0] for r in (0, 1)] == [31, 30]
+    for r in (0, 1):
+        assert np.array_equal(got[r][1], ref)
+
+
 def test_two_rank_token_sharding_matches_unsharded():
     from oracle import convrot_oracle as O
     from synthetic import CONFIGS, make_inputs

@@ -28,6 +28,29 @@ def strided(X: torch.Tensor, extra: int = 8) -> torch.Tensor:
     return buf[:, :K]
 
 
+CANARY = 0xA5          # guard byte around every code buffer
+SCALE_CANARY = -123.0  # guard value after the last scale
+
+
+def quant_guarded(fn, X, g, int8=False, extra=32):
+    """Run a rotate+quantise entry point into buffers with guard regions: code rows wider than
+    their defined K_pad / 2 (or K_pad) bytes, one guard row after the last, and guard scales
+    after sx[M - 1]. Asserts that the kernel wrote nothing outside the defined region and returns
+    (q, s) views of the defined outputs."""
+    M, K = X.shape
+    K_pad = O.padded_k(K, g)
+    row_bytes = K_pad if int8 else K_pad // 2
+    ldq = (row_bytes + extra + 15) // 16 * 16
+    qbuf = torch.full((M + 1, ldq), CANARY, dtype=torch.uint8, device="cuda")
+    sbuf = torch.full((M + 8,), SCALE_CANARY, dtype=torch.float32, device="cuda")
+    fn(X, g, qbuf[:M], sbuf[:M])
+    torch.cuda.synchronize()
+    assert (qbuf[:M, row_bytes:] == CANARY).all(), "bytes written past the defined code row"
+    assert (qbuf[M] == CANARY).all(), "bytes written past the last code row"
+    assert (sbuf[M:] == SCALE_CANARY).all(), "scales written past row M - 1"
+    return qbuf[:M, :row_bytes], sbuf[:M]
+
+
 def run_and_check(b, X_cpu, g, what, rows=None, weight=False):
     Xd = X_cpu.cuda()
     fn = b.prepack_weight if weight else b.rotate_quant_act
@@ -73,6 +96,43 @@ def test_quant_ragged_tiles(cuda_lib, g):
     ref_q, ref_s, ref_c = O.rotate_quant(bf16_to_f64(X), g)
     check_codes(gpu_codes(q, K_pad), ref_c, f"ragged g={g}")
     check_scales(s, ref_s, f"ragged g={g}")
+
+
+@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("int8", [False, True])
+@pytest.mark.parametrize("M,K", [(37, None), (300, None), (5, 8), (300, 1088), (300, 9280)])
+def test_quant_streamed_rows(cuda_lib, g, int8, M, K):
+    """K a multiple of 8 (whole rows stream through the shared ring): ragged K inside the last
+    group, row counts that are not a multiple of the rows per round, rows of 2 to 10240 padded
+    columns (K = 1088 and 9280 at g = 1024 pad 64 and 960 zero columns into the last group);
+    guard bytes around every output."""
+    if K is None:
+        K = 3 * g + 8
+    X = make_matrix(M, K, seed=M + K + g, row_outliers=min(3, M), row_scale=40.0)
+    fn = cuda_lib.rotate_quant_i8 if int8 else cuda_lib.rotate_quant_act
+    q, s = quant_guarded(fn, strided(X, extra=16), g, int8=int8)
+    K_pad = O.padded_k(K, g)
+    X64 = bf16_to_f64(X)
+    if int8:
+        ref_c, ref_s = O.rotate_quant_int8(X64, g)
+        got = q.cpu().numpy().view(np.int8)
+    else:
+        _, ref_s, ref_c = O.rotate_quant(X64, g)
+        got = gpu_codes(q, K_pad)
+    check_codes(got, ref_c, f"M={M} K={K} g={g} int8={int8}")
+    check_scales(s, ref_s, f"M={M} K={K} g={g} int8={int8}")
+
+
+@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("K", [3 * 64 + 3, 1001])
+def test_quant_register_path_guards(cuda_lib, g, K):
+    """K not a multiple of 8 (the register-resident kernel): the same guard regions."""
+    X = make_matrix(37, K, seed=K + g, row_outliers=3, row_scale=40.0)
+    q, s = quant_guarded(cuda_lib.rotate_quant_act, strided(X), g)
+    K_pad = O.padded_k(K, g)
+    _, ref_s, ref_c = O.rotate_quant(bf16_to_f64(X), g)
+    check_codes(gpu_codes(q, K_pad), ref_c, f"K={K} g={g}")
+    check_scales(s, ref_s, f"K={K} g={g}")
 
 
 @pytest.mark.parametrize("g", GROUPS)
@@ -149,11 +209,16 @@ FULL = [("qkv", 256), ("mlp_up", 256), ("proj_out", 1024),
 
 @pytest.mark.parametrize("name,g", FULL)
 def test_quant_full_size(cuda_lib, name, g):
-    """Full-size activations (all rows on the GPU, oracle on a row sample) and weights."""
+    """Full-size activations (all rows on the GPU and in the oracle) and weights (all rows on the
+    GPU, the oracle on a row sample)."""
     w = CONFIGS[name]
     X, W, _ = make_inputs(w)
     rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(w.M, size=min(w.M, 768), replace=False))
-    run_and_check(cuda_lib, X, g, f"{name} X g={g}", rows=rows)
+    # activations: every row against the oracle (the code-match bar is judged on all M x K_pad)
+    q, s = quant_guarded(cuda_lib.rotate_quant_act, X.cuda(), g)
+    K_pad = O.padded_k(w.K, g)
+    _, ref_s, ref_c = O.rotate_quant(bf16_to_f64(X), g)
+    check_codes(gpu_codes(q, K_pad), ref_c, f"{name} X g={g}")
+    check_scales(s, ref_s, f"{name} X g={g}")
     wrows = np.sort(rng.choice(w.N, size=min(w.N, 768), replace=False))
     run_and_check(cuda_lib, W, g, f"{name} W g={g}", rows=wrows, weight=True)
