@@ -117,7 +117,7 @@ def traffic_key(kernel_name: str):
         if k in kernel_name:
             return k
     m = (re.search(r"rht_quant_reg_kernel<\s*\d+,\s*(\d+)", kernel_name)       # <G, QM, ...>
-         or re.search(r"rht_quant_tma_kernel<\s*\d+,\s*\d+,\s*(\d+)", kernel_name))  # <G, TT, QM>
+         or re.search(r"rht_quant_ring_kernel<\s*\d+,\s*(\d+)", kernel_name))  # <G, QM>
     if m:   # code mode: 7 int4, 127 int8, 6 NVFP4, 5 MXFP4
         return {"7": "rht_quant_kernel", "127": "rht_quant_kernel_i8",
                 "6": "rht_quant_kernel_fp4", "5": "rht_quant_kernel_mx"}.get(m.group(1))
@@ -593,19 +593,34 @@ def main():
 
     def per_launch_ms(fn, operand_sets):
         """Average launch duration of one kernel: K launches back to back over rotating operand
-        copies, between two events."""
+        copies, between two events. The launches are captured once in a CUDA graph (each
+        operand copy in turn) and the graph is replayed: a single quantisation launch takes the
+        device less time than the Python binding takes the host to issue one call, so timing
+        launches issued one by one from Python would time the host."""
         n = len(operand_sets)
         for i in range(n):
             fn(operand_sets[i])
+        torch.cuda.synchronize()
+        per_graph = n * max(1, min(K, 200) // n)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(per_graph):
+                    fn(operand_sets[i % n])
+        torch.cuda.synchronize()
+        replays = max(1, -(-K // per_graph))
+        graph.replay()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        torch.cuda._sleep(PRIME_CYCLES)
         t0.record(stream)
-        for i in range(K):
-            fn(operand_sets[i % n])
+        for _ in range(replays):
+            graph.replay()
         t1.record(stream)
         torch.cuda.synchronize()
-        return slowest_rank_ms(t0.elapsed_time(t1)) / K
+        del graph
+        return slowest_rank_ms(t0.elapsed_time(t1)) / (replays * per_graph)
 
     # the quantisation alone touches far fewer bytes per launch than a step: rotate over more
     # copies of its operands (sharing the step's code and scale buffers)
@@ -783,8 +798,9 @@ def main():
         "quant_us": quant_avg * 1e3,
         "gemm_us": gemm_avg * 1e3,
         "kernel_times": "quant_us and gemm_us (and both rooflines): average launch duration "
-                        "of K launches of that kernel alone, back to back over rotating "
-                        "operand copies larger than L2, between two CUDA events",
+                        "of that kernel alone, launched back to back over rotating operand "
+                        "copies larger than L2 (captured once in a CUDA graph, replayed to at "
+                        "least K launches), between two CUDA events",
         "kernel_split": {"ms_per_step": ev_total_ms / K,
                          "quant_us": statistics.mean(ev_quant_ms) * 1e3,
                          "gemm_us": statistics.mean(ev_gemm_ms) * 1e3,

@@ -18,11 +18,10 @@
 //    chunks of a group (4 lanes of one warp): they swap 16-value blocks with three shuffle
 //    rounds (see the slot layout below). For G = 1024 (digits 3, 4 over 16 lanes) the lanes
 //    exchange their values once through an XOR-swizzled shared-memory tile.
-//  * Two kernels: a persistent register-resident kernel (direct 128-bit loads, the next row
-//    group's data prefetched into registers while the current one is transformed), used for
-//    every G <= 256 and any K; and, for G = 1024 with K a multiple of 64, a persistent kernel
-//    whose producer warp streams row groups into a shared-memory ring with 3-D TMA copies
-//    (long rows keep more bytes in flight that way).
+//  * The persistent register-resident kernel here (direct 128-bit loads, the next row group's
+//    data prefetched into registers while the current one is transformed) serves the shapes
+//    the row-streaming kernel of rht_quant_ring.cuh does not take (K not a multiple of 8, rows
+//    longer than 16384 columns) and the floating-point (NVFP4, MXFP4) modes.
 //  * The row absmax is combined across the row's threads with one shared-memory atomicMax
 //    (non-negative floats order like their bit patterns).
 //  * Rounding uses fma(v, inv, 1.5 * 2^23): the fp32 sum rounds v * inv to the nearest
@@ -631,168 +630,6 @@ __device__ __forceinline__ void blocks_1024(float (&v)[kChunk], float4* __restri
   __syncwarp();                     // loads complete before the next round's stores
 }
 
-// Persistent TMA-staged kernel (K a multiple of 64, K_pad <= 16384). A producer warp streams
-// groups of R rows into an S-deep shared-memory ring with one 3-D tensor copy per group
-// (box {64 elements, K_pad/64, R}, 128-byte swizzle, zero fill beyond K and M); compute
-// threads read their 64 elements from the ring without bank conflicts (16-byte chunk index
-// XOR (piece & 7)) while the next groups are in flight.
-// TT = compute threads per CTA (target). Rows with at most 128 pieces run 128-thread CTAs and
-// a producer warp, three per SM with a 3-deep ring (more independent CTAs hide the per-group
-// barrier). Longer rows run 256-thread CTAs, two per SM with a 1-deep ring and no producer warp:
-// thread 0 refills the slot once every warp has read it, so the next group loads while this
-// one is transformed, and an 8-warp CTA keeps 128 registers per thread (a ninth warp would
-// cap them at 96 and spill).
-template <int TT>
-constexpr int tma_min_blocks() {
-  return TT <= 128 ? 3 : 2;
-}
-template <int TT>
-__host__ __device__ constexpr int tma_ring_depth() {
-  return TT <= 128 ? 3 : 1;
-}
-template <int TT>
-__host__ __device__ constexpr bool tma_inline_producer() {
-  return TT > 128;
-}
-
-template <int G, int TT, int QM>
-__global__ void __launch_bounds__(TT + (tma_inline_producer<TT>() ? 0 : 32), tma_min_blocks<TT>())
-rht_quant_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int K_pad,
-                     uint8_t* __restrict__ Q, int64_t ldq, float* __restrict__ S, int R, int P,
-                     int64_t num_groups, int compute_threads) {
-  constexpr int kRingDepth = tma_ring_depth<TT>();
-  constexpr bool kInline = tma_inline_producer<TT>();
-  extern __shared__ __align__(1024) unsigned char smem_ring[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_ring) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int stage_bytes = R * K_pad * 2;                  // one group of R rows (bf16)
-  const int stage_pitch = (stage_bytes + 1023) & ~1023;
-  float4* xbuf = reinterpret_cast<float4*>(base + kRingDepth * stage_pitch);
-  unsigned int* amax_s = reinterpret_cast<unsigned int*>(
-      base + kRingDepth * stage_pitch + (G >= 256 ? compute_threads * 256 : 0));   // [3][R]
-  uint64_t* full = reinterpret_cast<uint64_t*>(amax_s + 3 * R + ((3 * R) & 1));
-  uint64_t* empty = full + kRingDepth;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kRingDepth);
-
-  const int tid = threadIdx.x;
-  const int compute_warps = compute_threads / 32;
-  const int pieces_per_row = K_pad / kChunk;
-  if (tid == 0) {
-    for (int i = 0; i < kRingDepth; ++i) {
-      mbar_init(full + i, 1);
-      mbar_init(empty + i, compute_warps);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  for (int i = tid; i < 3 * R; i += blockDim.x) amax_s[i] = 0u;
-  __syncthreads();
-  grid_dependency_wait();
-  launch_dependents();
-
-  if (!kInline && tid >= compute_threads) {
-    // ---------------------------------------------------------------- producer warp
-    if (tid == compute_threads) {
-      tma_prefetch_desc(&tmX);
-      int64_t i = 0;
-      for (int64_t rg = blockIdx.x; rg < num_groups; rg += gridDim.x, ++i) {
-        const int slot = static_cast<int>(i % kRingDepth);
-        if (i >= kRingDepth &&
-            !mbar_wait(empty + slot, static_cast<uint32_t>((i / kRingDepth) - 1) & 1, abort_flag))
-          break;
-        mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(stage_bytes));
-        tma_load_3d(base + slot * stage_pitch, &tmX, full + slot, 0, 0,
-                    static_cast<int32_t>(rg * R));
-      }
-      // drain: every issued copy has landed before the CTA can exit
-      const int64_t issued = i;
-      for (int64_t s = (issued > kRingDepth ? issued - kRingDepth : 0); s < issued; ++s) {
-        uint32_t polls = 0;
-        while (!mbar_try_wait(full + (s % kRingDepth), static_cast<uint32_t>(s / kRingDepth) & 1) &&
-               ++polls < kMaxPolls) {
-        }
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------------ compute threads
-  const int r_local = tid / P;
-  const int c = tid - r_local * P;
-  const bool lane_active = r_local < R;
-  const int p = r_local * pieces_per_row + c;            // this thread's 128-byte piece
-  int64_t issued = 0;                                    // inline producer: loads issued
-  if (kInline && tid == 0) {
-    tma_prefetch_desc(&tmX);
-    for (int s = 0; s < kRingDepth; ++s) {
-      const int64_t rg_s = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
-      if (rg_s >= num_groups) break;
-      mbar_arrive_expect_tx(full + s, static_cast<uint32_t>(stage_bytes));
-      tma_load_3d(base + s * stage_pitch, &tmX, full + s, 0, 0, static_cast<int32_t>(rg_s * R));
-      ++issued;
-    }
-  }
-  int64_t i = 0;
-  for (int64_t rg = blockIdx.x; rg < num_groups; rg += gridDim.x, ++i) {
-    const int slot = static_cast<int>(i % kRingDepth);
-    if (!mbar_wait(full + slot, static_cast<uint32_t>(i / kRingDepth) & 1, abort_flag)) break;
-    const int64_t row = rg * R + r_local;
-    const bool active = lane_active && row < M;
-    float v[kChunk];
-    {
-      const unsigned char* src = base + slot * stage_pitch + (lane_active ? p : 0) * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src + ((ch ^ (p & 7)) << 4));
-        bf16x2_to_f32(u.x, v[ch * 8 + 0], v[ch * 8 + 1]);
-        bf16x2_to_f32(u.y, v[ch * 8 + 2], v[ch * 8 + 3]);
-        bf16x2_to_f32(u.z, v[ch * 8 + 4], v[ch * 8 + 5]);
-        bf16x2_to_f32(u.w, v[ch * 8 + 6], v[ch * 8 + 7]);
-      }
-    }
-    // the ring slot may be refilled once every warp has read it (generic reads ordered
-    // before the asynchronous refill by the proxy fence)
-    fence_proxy_async_smem();
-    __syncwarp();
-    if ((tid & 31) == 0) mbar_arrive(empty + slot);
-    if (kInline && tid == 0) {
-      // refill the slot with this CTA's group kRingDepth rounds ahead once every warp has read
-      // it; a wait that gives up skips the load and every thread leaves at its next full wait
-      const int64_t rg_next = rg + static_cast<int64_t>(kRingDepth) * gridDim.x;
-      if (rg_next < num_groups &&
-          mbar_wait(empty + slot, static_cast<uint32_t>(i / kRingDepth) & 1, abort_flag)) {
-        mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(stage_bytes));
-        tma_load_3d(base + slot * stage_pitch, &tmX, full + slot, 0, 0,
-                    static_cast<int32_t>(rg_next * R));
-        ++issued;
-      }
-    }
-
-    transform_chunk<G>(v, xbuf, tid);
-    const float m = chunk_absmax(v);
-    unsigned int* am = amax_s + static_cast<int>(i % 3) * R;
-    if (active) atomicMax(am + r_local, __float_as_uint(m));
-    named_barrier_sync(1, compute_threads);
-    // the slot used by the previous group is no longer read by anyone: clear it for reuse
-    if (tid < R) amax_s[static_cast<int>((i + 2) % 3) * R + tid] = 0u;
-    if (active) {
-      float scale, inv;
-      row_scale<G, QM>(am[r_local], scale, inv);
-      if (c == 0) S[row] = scale;
-      store_row_codes<G, QM>(v, inv, Q + row * ldq, c, K_pad);
-    }
-  }
-  if (kInline && tid == 0) {
-    // after a wait gave up: every issued copy lands before the CTA can exit
-    for (int64_t s = i; s < issued; ++s) {
-      uint32_t polls = 0;
-      while (!mbar_try_wait(full + (s % kRingDepth), static_cast<uint32_t>(s / kRingDepth) & 1) &&
-             ++polls < kMaxPolls) {
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------------------------
 // Register-resident kernel: direct loads with a one-group prefetch, cross-thread digits by
 // warp shuffles (no shared-memory staging of the data).
@@ -1040,76 +877,12 @@ __global__ void make_rht_kernel(float* __restrict__ R, int G, int log4) {
   R[idx] = (eq & 1) ? -mag : mag;
 }
 
-using EncodeTiledFnQ = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFnQ encode_fn() {
-  static EncodeTiledFnQ fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnQ>(p);
-  }
-  return fn;
-}
-
 inline int sm_count() {
   int dev = 0, v = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
     return 148;
   return v;
-}
-
-// Returns cudaErrorNotSupported when the shape or the tensor map does not fit the TMA path.
-template <int G, int TT, int QM>
-cudaError_t launch_tma(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
-                       uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream) {
-  constexpr int kRingDepth = tma_ring_depth<TT>();
-  if (K % kChunk != 0 || K_pad / kChunk > 256) return cudaErrorNotSupported;
-  const int P = static_cast<int>(K_pad / kChunk);
-  int R = TT / P;
-  if (R < 1) R = 1;
-  const int compute_threads = ((R * P + 31) / 32) * 32;
-  if (compute_threads > TT) return cudaErrorNotSupported;
-  const int stage_pitch = (R * static_cast<int>(K_pad) * 2 + 1023) & ~1023;
-  const size_t smem = 1024 + static_cast<size_t>(kRingDepth) * stage_pitch +
-                      (G >= 256 ? static_cast<size_t>(compute_threads) * 256 : 0) +
-                      12 * static_cast<size_t>(R) + 8 + 2 * kRingDepth * 8 + 16;
-  if (smem > 227 * 1024) return cudaErrorNotSupported;
-  EncodeTiledFnQ enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tm;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kChunk), static_cast<cuuint64_t>(K / kChunk),
-                        static_cast<cuuint64_t>(M)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kChunk * 2), static_cast<cuuint64_t>(ldx * 2)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(P),
-                       static_cast<cuuint32_t>(R)};
-  cuuint32_t estr[3] = {1, 1, 1};
-  if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(X), dims, strides, box,
-          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorNotSupported;
-  auto kern = rht_quant_tma_kernel<G, TT, QM>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int64_t groups = (M + R - 1) / R;
-  int per_sm = 0;
-  const int threads = compute_threads + (tma_inline_producer<TT>() ? 0 : 32);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) !=
-          cudaSuccess || per_sm < 1)
-    per_sm = 1;
-  const int64_t slots = static_cast<int64_t>(sm_count()) * per_sm;
-  const int64_t grid = groups < slots ? groups : slots;
-  return launch_overlapped(kern, dim3(static_cast<unsigned>(grid)), dim3(threads),
-                           smem, stream, tm, M, static_cast<int>(K_pad), Q, ldq, S, R, P, groups,
-                           compute_threads);
 }
 
 template <int G, int QM, int kMaxT, int kMinBlocks>
@@ -1171,13 +944,6 @@ cudaError_t launch_g(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64
   // K a multiple of 8 and rows of at most 16384 columns: whole rows stream into a shared ring
   {
     const cudaError_t e = launch_ring<G, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream);
-    if (e != cudaErrorNotSupported) return e;
-  }
-  if constexpr (G == 1024) {
-    // long groups: the TMA-staged kernel when the row fits its ring (K a multiple of 64)
-    const cudaError_t e = (K_pad / kChunk <= 128)
-                              ? launch_tma<G, 128, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream)
-                              : launch_tma<G, 256, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream);
     if (e != cudaErrorNotSupported) return e;
   }
   // rows of up to 16384 columns: CTAs of at most 256 threads, two per SM; longer rows (at most
