@@ -54,10 +54,11 @@ def parse_args():
                    help="write profiles/ncu_traffic_<config>.json from ncu --csv captures "
                         "(comma-separated) of dram__bytes_read.sum and dram__bytes_write.sum, "
                         "then exit")
-    p.add_argument("--variant", default="w4a4", choices=("w4a4", "w8a8", "nvfp4", "mxfp4"),
+    p.add_argument("--variant", default="w4a4", choices=("w4a4", "w8a8", "nvfp4", "mxfp4", "fused"),
                    help="w4a4: the ConvLinear4bit layer (headline); w8a8: the int8 variant; "
                         "nvfp4: the floating-point (e2m1 + e4m3 block scales) variant; "
-                        "mxfp4: e2m1 with a power-of-two (e8m0) scale per 32 K")
+                        "mxfp4: e2m1 with a power-of-two (e8m0) scale per 32 K; fused: the W4A4 "
+                        "layer through its one-call entry point (codes in a caller workspace)")
     return p.parse_args()
 
 
@@ -68,6 +69,8 @@ def metric_name(variant="w4a4"):
         return "ConvRot MXFP4 layer TOPS and RHT+fp4-quant GB/s at FLUX-like M=4608 shapes"
     if variant == "w8a8":
         return "ConvRot W8A8 layer TOPS and RHT+int8-quant GB/s at FLUX-like M=4608 shapes"
+    if variant == "fused":
+        return "ConvLinear4bit (fused call) TOPS and RHT+int4-quant GB/s at FLUX-like M=4608 shapes"
     return "ConvLinear4bit TOPS and RHT+int4-quant GB/s at FLUX-like M=4608 shapes"
 
 
@@ -472,6 +475,7 @@ def main():
     Ml = X.shape[0]                               # token rows this rank runs per step
     Xd, Wd = X.to(dev), W.to(dev)
     int8 = args.variant == "w8a8"
+    fused = args.variant == "fused"
     mx = args.variant == "mxfp4"
     fp4 = mx or args.variant == "nvfp4"
     u8, f32, bf16 = torch.uint8, torch.float32, torch.bfloat16
@@ -522,7 +526,12 @@ def main():
             l_fn(st["qx"], st["sx"], st["qw"], st["sw"], K_pad, out=st["Y"])
 
         def layer(X_):
+            if fused:
+                return B.w4a4_linear_fused(X_, qw0, sw0, g)
             return layer_fn(X_, qw0, sw0, g, K_pad)
+
+        def step_fused(st):
+            B.w4a4_linear_fused(st["X"], st["qw"], st["sw"], g, out=st["Y"], workspace=st["ws"])
 
     def new_set():
         st = {"X": Xd.clone(), "qx": torch.empty(Ml, ldq, dtype=u8, device=dev),
@@ -535,6 +544,8 @@ def main():
                 st["gw"] = gw0.clone()
         else:
             st["sw"] = sw0.clone()
+        if fused:
+            st["ws"] = torch.empty(B.fused_workspace_bytes(Ml, w.K, g), dtype=u8, device=dev)
         return st
 
     # L2 policy: inputs larger than L2 instead of a flush inside the timed region. Each step
@@ -546,9 +557,15 @@ def main():
     sets += [new_set() for _ in range(n_sets - 1)]
     stream = torch.cuda.current_stream()
 
+    def step(st):
+        if fused:
+            step_fused(st)
+        else:
+            quant(st)
+            linear(st)
+
     for i in range(max(args.warmup, n_sets)):
-        quant(sets[i % n_sets])
-        linear(sets[i % n_sets])
+        step(sets[i % n_sets])
     torch.cuda.synchronize()
     assert B.device_status() == 0
     if strong:
@@ -574,11 +591,12 @@ def main():
         t0.record(stream)
         for i in range(K):
             st = sets[i % n_sets]
-            if kernel_events:
-                ev[i][0].record(stream)
+            if not kernel_events:
+                step(st)
+                continue
+            ev[i][0].record(stream)
             quant(st)
-            if kernel_events:
-                ev[i][1].record(stream)
+            ev[i][1].record(stream)
             linear(st)
         t1.record(stream)
         torch.cuda.synchronize()
@@ -633,9 +651,16 @@ def main():
     with ClockSampler(local_rank) as clk:
         t_wall0 = time.time()
         total_ms, _, _ = timed_run(kernel_events=False)          # the headline: K plain steps
-        ev_total_ms, ev_quant_ms, ev_gemm_ms = timed_run(kernel_events=True)
-        quant_ms = per_launch_ms(quant, q_sets)
-        gemm_ms = per_launch_ms(linear, sets)
+        if fused:
+            # the fused call's two kernels are not separable by events between calls: the GEMM's
+            # time is the fused call's minus its quantisation's, each timed alone
+            ev_total_ms = ev_quant_ms = ev_gemm_ms = None
+            quant_ms = per_launch_ms(quant, q_sets)
+            gemm_ms = per_launch_ms(step_fused, sets) - quant_ms
+        else:
+            ev_total_ms, ev_quant_ms, ev_gemm_ms = timed_run(kernel_events=True)
+            quant_ms = per_launch_ms(quant, q_sets)
+            gemm_ms = per_launch_ms(linear, sets)
         t_wall1 = time.time()
     del q_sets
     ms_per_step = total_ms / K
@@ -801,12 +826,12 @@ def main():
                         "of that kernel alone, launched back to back over rotating operand "
                         "copies larger than L2 (captured once in a CUDA graph, replayed to at "
                         "least K launches), between two CUDA events",
-        "kernel_split": {"ms_per_step": ev_total_ms / K,
-                         "quant_us": statistics.mean(ev_quant_ms) * 1e3,
-                         "gemm_us": statistics.mean(ev_gemm_ms) * 1e3,
-                         "how": "a second run of K steps with CUDA events between the two "
-                                "kernels of every step (each event drains the stream, so "
-                                "these times include that drain)"},
+        "kernel_split": None if fused else {
+            "ms_per_step": ev_total_ms / K,
+            "quant_us": statistics.mean(ev_quant_ms) * 1e3,
+            "gemm_us": statistics.mean(ev_gemm_ms) * 1e3,
+            "how": "a second run of K steps with CUDA events between the two kernels of every "
+                   "step (each event drains the stream, so these times include that drain)"},
         "roofline": {"bound": "tensor", "kernel": gemm_kernel,
                      "achieved": ops / (gemm_avg / 1e3) / 1e12,
                      "peak": int8_peak, "unit": "TFLOP/s",

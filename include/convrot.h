@@ -265,6 +265,29 @@ int convrot_mxfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
                            int64_t ldqw, const uint8_t* sfw, float* acc, int64_t ldacc, int64_t M,
                            int64_t N, int64_t K4, convrot_stream_t stream);
 
+/* ---- The whole layer in one call ---------------------------------------------------------
+ * "ConvRot" paper, Abstract and Fig. 3: ConvLinear4bit is a plug-and-play module that
+ * integrates rotation, quantisation, GEMM and dequantisation. One call computes, from the bf16
+ * activations, exactly what convrot_rotate_quant_act followed by convrot_w4a4_linear computes
+ * (the same codes, scales and output formula):
+ *   Y[m,n] = bf16_rne((float(acc[m,n]) * sx[m]) * sw[n] + float(bias[n]))
+ * The packed activation codes and their scales live in the caller's workspace for the
+ * duration of the call (contents undefined afterwards; nothing else may use it while the call
+ * runs on the GPU).
+ *   X: bf16 [M, ldx]; qw, sw, bias: as for convrot_w4a4_linear (qw from
+ *   convrot_prepack_weight with the same group); Y: bf16 [M, ldy], ldy >= N.
+ *   workspace: device, 256-byte aligned, at least convrot_w4a4_fused_workspace_bytes(M, K,
+ *   group) bytes (packed codes [M, round_up(K_pad / 2, 16)], then the row scales).
+ * Limits: 0 < K, K_pad <= 32768, M, N < 2^31. Alignment: X 16-byte aligned with ldx a multiple
+ * of 8; qw, Y, bias, sw as for convrot_w4a4_linear. M == 0 or N == 0 is a no-op.
+ * Errors: INVALID_GROUP, SHAPE, NULL, ALIGN, DEVICE, CUDA. */
+int64_t convrot_w4a4_fused_workspace_bytes(int64_t M, int64_t K, int group);
+
+int convrot_w4a4_linear_fused(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int group,
+                              const uint8_t* qw, int64_t ldqw, const float* sw,
+                              const uint16_t* bias, uint16_t* Y, int64_t ldy, int64_t N,
+                              void* workspace, int64_t workspace_bytes, convrot_stream_t stream);
+
 /* Test export of the failure path: launches one warp that waits on a barrier nothing arrives
  * on, gives up after `polls` polls (1 .. 2^24; each poll suspends for a hardware-chosen time
  * window) and records CONVROT_ERR_TIMEOUT in the device status word, exactly as a kernel's

@@ -59,6 +59,10 @@ _SIGNATURES = {
                               _c_i64, _c_i64, _c_i64, _c_i64, _c_ptr], _c_int),
     "convrot_mxfp4_gemm_f32": ([_c_ptr, _c_i64, _c_ptr, _c_ptr, _c_i64, _c_ptr, _c_ptr, _c_i64,
                                 _c_i64, _c_i64, _c_i64, _c_ptr], _c_int),
+    "convrot_w4a4_fused_workspace_bytes": ([_c_i64, _c_i64, _c_int], _c_i64),
+    "convrot_w4a4_linear_fused": ([_c_ptr, _c_i64, _c_i64, _c_i64, _c_int, _c_ptr, _c_i64, _c_ptr,
+                                   _c_ptr, _c_ptr, _c_i64, _c_i64, _c_ptr, _c_i64, _c_ptr],
+                                  _c_int),
     "convrot_selftest_bounded_wait": ([_c_int, _c_ptr], _c_int),
     "convrot_device_status": ([ctypes.POINTER(_c_int), _c_int], _c_int),
 }
@@ -337,6 +341,37 @@ def conv_linear_mxfp4(X, qw, sfw, group: int, bias=None):
     """The MXFP4 variant's forward on prepacked weights."""
     qx, sfx = rotate_quant_act_mxfp4(X, group)
     return mxfp4_linear(qx, sfx, qw, sfw, nvfp4_k(X.shape[1], group), bias=bias)
+
+
+def fused_workspace_bytes(M: int, K: int, group: int) -> int:
+    """Bytes of device workspace w4a4_linear_fused needs for an [M, K] activation."""
+    v = lib.convrot_w4a4_fused_workspace_bytes(int(M), int(K), int(group))
+    if v < 0:
+        raise ConvRotError("convrot_w4a4_fused_workspace_bytes", 1 if group not in GROUPS else 2)
+    return int(v)
+
+
+def w4a4_linear_fused(X, qw, sw, group: int, bias=None, out=None, workspace=None):
+    """The whole ConvLinear4bit layer in one call: bf16 X [M, K] -> bf16 Y [M, N] (the same
+    result as rotate_quant_act followed by w4a4_linear). `workspace` (uint8 device tensor of at
+    least fused_workspace_bytes(M, K, group) bytes, 256-byte aligned) is allocated here with
+    torch when not given."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a 2-D bf16 tensor with unit column stride")
+    M, K = X.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    need = fused_workspace_bytes(M, K, group)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _check("convrot_w4a4_linear_fused",
+           lib.convrot_w4a4_linear_fused(_ptr(X), M, K, X.stride(0), int(group), _ptr(qw),
+                                         qw.stride(0), _ptr(sw), _ptr(bias), _ptr(out),
+                                         out.stride(0), N, _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream()))
+    return out
 
 
 def selftest_bounded_wait(polls: int = 1 << 16):

@@ -181,6 +181,16 @@ int rotate_quant_mx(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int gr
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// The fused layer's workspace: packed activation codes [M, round_up(K_pad / 2, 16)], then the
+// row scales at the next 256-byte boundary.
+int64_t fused_codes_ld(int64_t K_pad) { return (K_pad / 2 + 15) / 16 * 16; }
+int64_t fused_scales_offset(int64_t M, int64_t K_pad) {
+  return (M * fused_codes_ld(K_pad) + 255) / 256 * 256;
+}
+int64_t fused_workspace_bytes(int64_t M, int64_t K_pad) {
+  return fused_scales_offset(M, K_pad) + (M * 4 + 255) / 256 * 256;
+}
+
 }  // namespace
 }  // namespace convrot
 
@@ -383,6 +393,39 @@ int convrot_mxfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
   return from_cuda(launch_nvfp4_gemm(qx, ldqx, sfx, nullptr, qw, ldqw, sfw, nullptr, nullptr, acc,
                                      ldacc, M, N, K4, GemmOut::kRawS32,
                                      reinterpret_cast<cudaStream_t>(stream), true));
+}
+
+int64_t convrot_w4a4_fused_workspace_bytes(int64_t M, int64_t K, int group) {
+  if (!valid_group(group) || K < 0 || M < 0) return -1;
+  return fused_workspace_bytes(M, (K + group - 1) / group * group);
+}
+
+int convrot_w4a4_linear_fused(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int group,
+                              const uint8_t* qw, int64_t ldqw, const float* sw,
+                              const uint16_t* bias, uint16_t* Y, int64_t ldy, int64_t N,
+                              void* workspace, int64_t workspace_bytes, convrot_stream_t stream) {
+  if (!valid_group(group)) return CONVROT_ERR_INVALID_GROUP;
+  if (M < 0 || N < 0 || K < 0) return CONVROT_ERR_SHAPE;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  if (K == 0) return CONVROT_ERR_SHAPE;
+  if (workspace == nullptr) return CONVROT_ERR_NULL;
+  const int64_t K_pad = (K + group - 1) / group * group;
+  const int64_t ldq = fused_codes_ld(K_pad);
+  uint8_t* qx = static_cast<uint8_t*>(workspace);
+  float* sx = reinterpret_cast<float*>(qx + fused_scales_offset(M, K_pad));
+  int st = check_quant_args(X, M, K, ldx, group, qx, ldq, sx, false);
+  if (st != CONVROT_OK) return st;
+  if ((st = gemm_args(qx, ldq, qw, ldqw, Y, ldy, M, N, K_pad, false)) != CONVROT_OK) return st;
+  if (workspace_bytes < fused_workspace_bytes(M, K_pad)) return CONVROT_ERR_SHAPE;
+  if (!aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
+  if (sw == nullptr) return CONVROT_ERR_NULL;
+  if (!aligned(sw, 4) || !aligned(bias, 2) || !aligned(Y, 2)) return CONVROT_ERR_ALIGN;
+  if ((st = check_device()) != CONVROT_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_rht_quant(X, M, K, ldx, group, qx, ldq, sx, cs, 7) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  return from_cuda(launch_w4a4_gemm(qx, ldq, sx, qw, ldqw, sw, bias, Y, ldy, M, N, K_pad,
+                                    GemmOut::kDequantBf16, cs));
 }
 
 int convrot_selftest_bounded_wait(int polls, convrot_stream_t stream) {

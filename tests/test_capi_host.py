@@ -31,7 +31,7 @@ def header_names():
 
 def test_library_exports_every_declared_symbol(b):
     names = header_names()
-    assert len(names) == 23
+    assert len(names) == 25
     assert b.exported_names() == names
     for n in names:
         assert hasattr(b.lib, n), n
@@ -192,3 +192,30 @@ def test_binding_fails_loudly_without_the_library(b, monkeypatch, tmp_path):
     monkeypatch.setattr(b._build, "LIBPATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError, match="not built"):
         b._load()
+
+
+def fused(b, X=FAKE, M=4, K=64, ldx=64, g=16, qw=FAKE, ldqw=32, sw=FAKE, bias=None, Y=FAKE,
+          ldy=64, N=64, ws=FAKE, wsb=None):
+    if wsb is None:
+        wsb = b.lib.convrot_w4a4_fused_workspace_bytes(M, K, g) if g in (16, 64, 256, 1024) else 0
+    return b.lib.convrot_w4a4_linear_fused(X, M, K, ldx, g, qw, ldqw, sw, bias, Y, ldy, N, ws,
+                                           wsb, None)
+
+
+def test_fused_workspace_and_argument_validation(b):
+    # packed codes [M, round_up(K_pad / 2, 16)], then the row scales at the next 256-byte boundary
+    ws = b.lib.convrot_w4a4_fused_workspace_bytes
+    assert ws(4, 64, 16) == 256 + 256
+    assert ws(4608, 3072, 256) == 4608 * 1536 + 4608 * 4 // 256 * 256
+    assert ws(37, 3000, 1024) == -(-37 * 1536 // 256) * 256 + 256
+    assert ws(4, 64, 48) == -1 and ws(-1, 64, 16) == -1
+    assert fused(b, g=48) == 1
+    assert fused(b, K=0) == 2
+    assert fused(b, K=40000, ldx=40000, ldqw=20480) == 2  # K_pad above the quantisation limit
+    assert fused(b, wsb=100) == 2                         # workspace too small
+    assert fused(b, ws=FAKE + 16) == 4                    # workspace not 256-byte aligned
+    assert fused(b, X=FAKE + 2) == 4 and fused(b, ldx=68) == 4
+    assert fused(b, X=None) == 3 and fused(b, sw=None) == 3 and fused(b, qw=None) == 3
+    assert fused(b, ws=None) == 3
+    assert fused(b, ldy=32) == 2                          # ldy < N
+    assert fused(b, M=0) == 0 and fused(b, N=0) == 0      # no-ops, nothing touched
