@@ -288,6 +288,35 @@ int convrot_w4a4_linear_fused(const uint16_t* X, int64_t M, int64_t K, int64_t l
                               const uint16_t* bias, uint16_t* Y, int64_t ldy, int64_t N,
                               void* workspace, int64_t workspace_bytes, convrot_stream_t stream);
 
+/* Size of the library's built-in scratch array used by convrot_w4a4_linear_fused_noalloc. */
+#define CONVROT_NOALLOC_SCRATCH_BYTES (8 * 1024 * 1024)
+
+/* The one-call layer for callers that cannot allocate device memory. Nothing in the paper
+ * corresponds to this entry point: it exists for callers that are handed streams and tensors
+ * but cannot obtain memory of their own at call time -- for example code that runs while a
+ * stream is being captured into a CUDA graph (cudaMalloc is not a stream operation and is not
+ * allowed during such a capture), or a plugin inside another runtime that owns the allocator and
+ * gives the plugin no workspace. It computes exactly what convrot_w4a4_linear_fused computes,
+ * with the same arguments except the workspace: the packed codes and scales go to a fixed
+ * scratch array of CONVROT_NOALLOC_SCRATCH_BYTES (8 MiB) that the library holds in device
+ * memory on every GPU where it is loaded, until the process exits. The call allocates nothing.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress),
+ *    with that device current; make that first call before any stream capture begins.
+ *  - Every call on a device uses the same array. Calls whose work overlaps on the GPU (on two
+ *    streams, or from two host threads) race on it and give undefined results; calls that follow
+ *    each other in one stream are safe. The array keeps the last call's contents; nothing in it
+ *    needs to start at zero (each call writes every byte it reads).
+ *  - Shapes whose workspace (convrot_w4a4_fused_workspace_bytes(M, K, group)) exceeds the array
+ *    are rejected with CONVROT_ERR_SHAPE before anything runs; e.g. M = 4608 tokens fit for
+ *    K_pad <= 3584 (FLUX's QKV and MLP-up activations, K = 3072), any M <= 512 for
+ *    K_pad <= 16384.
+ * Other limits, alignment rules and errors as convrot_w4a4_linear_fused; CONVROT_ERR_CUDA also
+ * reports a failed address lookup. */
+int convrot_w4a4_linear_fused_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
+                                      int group, const uint8_t* qw, int64_t ldqw, const float* sw,
+                                      const uint16_t* bias, uint16_t* Y, int64_t ldy, int64_t N,
+                                      convrot_stream_t stream);
+
 /* Test export of the failure path: launches one warp that waits on a barrier nothing arrives
  * on, gives up after `polls` polls (1 .. 2^24; each poll suspends for a hardware-chosen time
  * window) and records CONVROT_ERR_TIMEOUT in the device status word, exactly as a kernel's

@@ -63,6 +63,9 @@ _SIGNATURES = {
     "convrot_w4a4_linear_fused": ([_c_ptr, _c_i64, _c_i64, _c_i64, _c_int, _c_ptr, _c_i64, _c_ptr,
                                    _c_ptr, _c_ptr, _c_i64, _c_i64, _c_ptr, _c_i64, _c_ptr],
                                   _c_int),
+    "convrot_w4a4_linear_fused_noalloc": ([_c_ptr, _c_i64, _c_i64, _c_i64, _c_int, _c_ptr,
+                                           _c_i64, _c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64,
+                                           _c_ptr], _c_int),
     "convrot_selftest_bounded_wait": ([_c_int, _c_ptr], _c_int),
     "convrot_device_status": ([ctypes.POINTER(_c_int), _c_int], _c_int),
 }
@@ -371,6 +374,27 @@ def w4a4_linear_fused(X, qw, sw, group: int, bias=None, out=None, workspace=None
                                          out.stride(0), N, _ptr(workspace),
                                          workspace.numel() * workspace.element_size(),
                                          _stream()))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def w4a4_linear_fused_noalloc(X, qw, sw, group: int, bias=None, out=None):
+    """The one-call layer with the library's built-in scratch array instead of a workspace
+    (for callers that cannot allocate device memory; see convrot_w4a4_linear_fused_noalloc in
+    include/convrot.h for the size limit and the rule that overlapping calls race). Allocates
+    only `out` (with torch) when it is not given."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a 2-D bf16 tensor with unit column stride")
+    M, K = X.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    _check("convrot_w4a4_linear_fused_noalloc",
+           lib.convrot_w4a4_linear_fused_noalloc(_ptr(X), M, K, X.stride(0), int(group), _ptr(qw),
+                                                 qw.stride(0), _ptr(sw), _ptr(bias), _ptr(out),
+                                                 out.stride(0), N, _stream()))
     return out
 
 

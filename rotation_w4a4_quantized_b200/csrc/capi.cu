@@ -5,6 +5,7 @@
 // launches on the caller's stream. It allocates no memory.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/convrot.h"
@@ -15,6 +16,11 @@
 #include "w4a4_gemm.cuh"
 #include "w8a8_gemm.cuh"
 #include "nvfp4_gemm.cuh"
+
+// Scratch of convrot_w4a4_linear_fused_noalloc (the packed activation codes and row scales of
+// one call): a fixed device array, so that the call allocates nothing. Every GPU that loads the
+// library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CONVROT_NOALLOC_SCRATCH_BYTES];
 
 namespace convrot {
 namespace {
@@ -189,6 +195,30 @@ int64_t fused_scales_offset(int64_t M, int64_t K_pad) {
 }
 int64_t fused_workspace_bytes(int64_t M, int64_t K_pad) {
   return fused_scales_offset(M, K_pad) + (M * 4 + 255) / 256 * 256;
+}
+
+// The device address of the no-alloc scratch array (below), looked up once per device: in host
+// code the array's name is only a host-side stand-in, never a device address.
+constexpr int64_t kNoAllocScratchBytes = CONVROT_NOALLOC_SCRATCH_BYTES;
+std::atomic<void*> g_noalloc_scratch_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up on first use).
+int noalloc_scratch(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return CONVROT_ERR_DEVICE;
+  }
+  void* p = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return CONVROT_ERR_CUDA;
+    }
+    g_noalloc_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  *addr = p;
+  return CONVROT_OK;
 }
 
 }  // namespace
@@ -426,6 +456,24 @@ int convrot_w4a4_linear_fused(const uint16_t* X, int64_t M, int64_t K, int64_t l
     return CONVROT_ERR_CUDA;
   return from_cuda(launch_w4a4_gemm(qx, ldq, sx, qw, ldqw, sw, bias, Y, ldy, M, N, K_pad,
                                     GemmOut::kDequantBf16, cs));
+}
+
+int convrot_w4a4_linear_fused_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
+                                      int group, const uint8_t* qw, int64_t ldqw, const float* sw,
+                                      const uint16_t* bias, uint16_t* Y, int64_t ldy, int64_t N,
+                                      convrot_stream_t stream) {
+  if (!valid_group(group)) return CONVROT_ERR_INVALID_GROUP;
+  if (M < 0 || N < 0 || K < 0) return CONVROT_ERR_SHAPE;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  // larger than the built-in scratch array: rejected before anything is looked up or launched
+  if (fused_workspace_bytes(M, (K + group - 1) / group * group) > kNoAllocScratchBytes)
+    return CONVROT_ERR_SHAPE;
+  int st = check_device();
+  if (st != CONVROT_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != CONVROT_OK) return st;
+  return convrot_w4a4_linear_fused(X, M, K, ldx, group, qw, ldqw, sw, bias, Y, ldy, N, scratch,
+                                   kNoAllocScratchBytes, stream);
 }
 
 int convrot_selftest_bounded_wait(int polls, convrot_stream_t stream) {
