@@ -101,16 +101,6 @@ __device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) 
   hi = __uint_as_float(w & 0xFFFF0000u);
 }
 
-// Integer codes of v0 * inv and v1 * inv rounded half-to-even (|v * inv| <= 7.x, far below
-// 2^22), with one packed fma: the fp32 sum v * inv + 1.5 * 2^23 rounds v * inv to an integer in
-// one step, and the integer sits in the low mantissa bits.
-__device__ __forceinline__ void round_code2(float v0, float v1, float inv, int& q0, int& q1) {
-  const float2 r = __ffma2_rn(make_float2(v0, v1), make_float2(inv, inv),
-                              make_float2(12582912.0f, 12582912.0f));
-  q0 = __float_as_int(r.x) - 0x4B400000;
-  q1 = __float_as_int(r.y) - 0x4B400000;
-}
-
 // Four int8 codes of v[0..3] * inv -> one 32-bit word, code 0 in byte 0. The rounded sum's bit
 // pattern is 0x4B400000 + q, so its low byte is already q in two's complement (|q| <= 127:
 // |v| <= absmax and absmax * inv exceeds 127 by a few ulp at most, so no code saturates).
@@ -123,17 +113,6 @@ __device__ __forceinline__ uint32_t code_bytes4(float v0, float v1, float v2, fl
   const uint32_t lo = __byte_perm(__float_as_uint(r01.x), __float_as_uint(r01.y), 0x0040);
   const uint32_t hi = __byte_perm(__float_as_uint(r23.x), __float_as_uint(r23.y), 0x0040);
   return __byte_perm(lo, hi, 0x5410);
-}
-
-// Four codes -> 16 bits, code 0 in bits 0..3.
-__device__ __forceinline__ uint32_t pack4(int q0, int q1, int q2, int q3) {
-  uint32_t r;
-  asm("{\n\t.reg .u32 t;\n\t"
-      "cvt.pack.sat.s4.s32.b32 t, %4, %3, 0;\n\t"
-      "cvt.pack.sat.s4.s32.b32 %0, %2, %1, t;\n\t}"
-      : "=r"(r)
-      : "r"(q0), "r"(q1), "r"(q2), "r"(q3));
-  return r & 0xFFFFu;
 }
 
 // Eight codes of v[0..7] * inv (rounded half-to-even) -> one word, code i in bits 4i .. 4i+3.
@@ -234,15 +213,20 @@ __device__ __forceinline__ void store_codes(const float (&v)[kChunk], float inv,
       }
     }
   } else {
+    // 4 consecutive codes per a (16 bits at byte 32 a + 2 j of the group's 512 bytes): the low
+    // nibbles of the rounded sums' bit patterns, gathered by byte permutes as in code_nibbles8
     const int j = c & 15;
-    const int q_grp = c >> 4;
+    uint8_t* qg = qr + (c >> 4) * 512 + 2 * j;
+    const float2 m = make_float2(12582912.0f, 12582912.0f);
+    const float2 ii = make_float2(inv, inv);
 #pragma unroll
     for (int a = 0; a < 16; ++a) {
-      int q0, q1, q2, q3;
-      round_code2(v[a * 4 + 0], v[a * 4 + 1], inv, q0, q1);
-      round_code2(v[a * 4 + 2], v[a * 4 + 3], inv, q2, q3);
-      const uint32_t h = pack4(q0, q1, q2, q3);
-      *reinterpret_cast<uint16_t*>(qr + q_grp * 512 + a * 32 + 2 * j) = static_cast<uint16_t>(h);
+      const float2 r01 = __ffma2_rn(make_float2(v[a * 4 + 0], v[a * 4 + 1]), ii, m);
+      const float2 r23 = __ffma2_rn(make_float2(v[a * 4 + 2], v[a * 4 + 3]), ii, m);
+      const uint32_t e = __byte_perm(__float_as_uint(r01.x), __float_as_uint(r23.x), 0x0040);
+      const uint32_t o = __byte_perm(__float_as_uint(r01.y), __float_as_uint(r23.y), 0x0040);
+      *reinterpret_cast<uint16_t*>(qg + a * 32) =
+          static_cast<uint16_t>((e & 0x0F0Fu) | ((o << 4) & 0xF0F0u));
     }
   }
 }

@@ -191,6 +191,91 @@ __device__ __forceinline__ void lds_chunk(const unsigned char* __restrict__ src,
     }
 }
 
+// Shared-memory 16-byte loads and stores at explicit shared-window addresses. The ring and the
+// exchange rows are laid out so that every address a thread needs is a per-round (or
+// per-kernel) base XOR a compile-time constant, one logic instruction per access.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(a)
+               : "memory");
+  return r;
+}
+
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(a)
+               : "memory");
+  return r;
+}
+
+__device__ __forceinline__ void sts128f(uint32_t a, float x, float y, float z, float w) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z),
+               "f"(w)
+               : "memory");
+}
+
+// lds_chunk with the chunk at shared address src (128-byte aligned, so the unit index sits in
+// address bits 4..6 and the permutations are XORs of the address).
+template <int G>
+__device__ __forceinline__ void lds_chunk_sa(uint32_t src, int j, int perm, float (&v)[kChunk]) {
+  const uint32_t base = (G == 1024) ? (src | (static_cast<uint32_t>(perm) << 4))
+                                    : (src | (static_cast<uint32_t>(j) << 5));
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      // G = 1024: unit (2 s + h) ^ perm; G <= 256: unit 2 (s ^ j) + h
+      const uint32_t a = (G == 1024) ? (base ^ static_cast<uint32_t>((2 * s + h) << 4))
+                                     : ((base ^ static_cast<uint32_t>(s << 5)) + 16 * h);
+      const uint4 u = lds128(a);
+      float* d = v + 16 * s + 8 * h;
+      bf16x2_to_f32(u.x, d[0], d[1]);
+      bf16x2_to_f32(u.y, d[2], d[3]);
+      bf16x2_to_f32(u.z, d[4], d[5]);
+      bf16x2_to_f32(u.w, d[6], d[7]);
+    }
+}
+
+// transform_chunk<1024> with the exchange rows at shared address xb (this team's rows, 256-byte
+// aligned; thread tt owns the 256 bytes at xb + 256 tt). Same arithmetic and layouts.
+__device__ __forceinline__ void transform_chunk_1024_sa(float (&v)[kChunk], uint32_t xb, int tt,
+                                                        int perm) {
+  radix4_stage<1>(v);
+  radix4_stage<4>(v);
+  radix4_stage<16>(v);
+  // row tt, 16-byte piece ch ^ perm ^ (tt & 7): base | (wx << 4), XOR (ch << 4)
+  const uint32_t wbase = (xb + 256u * static_cast<uint32_t>(tt)) |
+                         (static_cast<uint32_t>(perm ^ (tt & 7)) << 4);
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch)
+    sts128f(wbase ^ static_cast<uint32_t>(ch << 4), v[4 * ch], v[4 * ch + 1], v[4 * ch + 2],
+            v[4 * ch + 3]);
+  __syncwarp();
+  // thread j takes piece j of rows t0 + a (a = 0..15) at piece position j ^ (a & 7)
+  const int j = tt & 15;
+  const uint32_t rbase = xb + 256u * static_cast<uint32_t>(tt & ~15) + (static_cast<uint32_t>(j) << 4);
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const uint32_t ra = rbase ^ static_cast<uint32_t>(a << 4);
+    const float4 w0 = lds128f(ra + 256u * a);
+    const float4 w1 = lds128f(ra + 256u * (a + 8));
+    v[a * 4 + 0] = w0.x;
+    v[a * 4 + 1] = w0.y;
+    v[a * 4 + 2] = w0.z;
+    v[a * 4 + 3] = w0.w;
+    v[(a + 8) * 4 + 0] = w1.x;
+    v[(a + 8) * 4 + 1] = w1.y;
+    v[(a + 8) * 4 + 2] = w1.z;
+    v[(a + 8) * 4 + 3] = w1.w;
+  }
+  radix4_stage<4>(v);   // digit 3 = a bits 0..1
+  radix4_stage<16>(v);  // digit 4 = a bits 2..3
+}
+
 // Codes of one chunk in the slot layout for G <= 64 (slot s holds columns 64 c + 16 (s ^ j) + e);
 // blocks at or past K_pad (ragged last chunk, G = 16) are not stored.
 template <int QM>
@@ -219,13 +304,15 @@ template <int G, int QM>
 __global__ void __launch_bounds__(32 * (kRingMaxWarps + 1), 1)
 rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t ldx, int K_pad,
                       uint8_t* __restrict__ Q, int64_t ldq, float* __restrict__ S, RingPlan pl) {
-  extern __shared__ __align__(128) unsigned char smem_rows[];
-  unsigned char* ring = smem_rows;
+  extern __shared__ __align__(1024) unsigned char smem_raw_rows[];
+  // 1024-byte aligned base (the plan reserves the slack)
+  unsigned char* smem_rows = smem_raw_rows + ((1024u - (smem_u32(smem_raw_rows) & 1023u)) & 1023u);
   const int team_threads = pl.team_warps * 32;
   const int ring_bytes = pl.slots * pl.slot_bytes;
   const int xbuf_bytes = (G == 1024) ? pl.teams * team_threads * 256 : 0;
-  float4* xbuf_all = reinterpret_cast<float4*>(ring + ring_bytes);
-  unsigned int* amax = reinterpret_cast<unsigned int*>(ring + ring_bytes + xbuf_bytes);
+  // exchange rows first (256-byte aligned rows), then the ring (128-byte aligned slots)
+  unsigned char* ring = smem_rows + xbuf_bytes;
+  unsigned int* amax = reinterpret_cast<unsigned int*>(ring + ring_bytes);
   const int amax_words = pl.teams * 3 * pl.TR;
   uint64_t* full = reinterpret_cast<uint64_t*>(amax + ((amax_words + 1) & ~1));
   uint64_t* empty = full + pl.slots;
@@ -306,7 +393,8 @@ rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t 
   const int j = tt & 3;                                   // slot layout (G <= 256)
   const int perm = tt & 7;                                // unit permutation (G = 1024)
   unsigned int* am_team = amax + team * 3 * pl.TR;
-  float4* xbuf = xbuf_all + team * team_threads * 16;
+  const uint32_t xbuf_sa = smem_u32(smem_rows) + 256u * static_cast<uint32_t>(team * team_threads);
+  const uint32_t ring_sa = smem_u32(ring);
   const int bar_id = 1 + team;
   const int chunk_off = (lane_ok ? r_local * pl.pitch : 0) + c * 128;
   // the lanes of this warp that hold the same row (a warp holds parts of up to 32 rows): their
@@ -321,7 +409,8 @@ rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t 
     const bool ok = wait_slot_claimed(seq + slot, k, abort_flag) &&
                     mbar_wait_backoff(full + slot, phase, abort_flag);
     float v[kChunk];
-    lds_chunk<G>(ring + slot * pl.slot_bytes + chunk_off, j, perm, v);
+    lds_chunk_sa<G>(ring_sa + static_cast<uint32_t>(slot * pl.slot_bytes + chunk_off), j, perm,
+                    v);
     // the slot may be refilled once every warp of the team has read it (generic reads ordered
     // before the asynchronous refill by the proxy fence)
     fence_proxy_async_smem();
@@ -329,7 +418,7 @@ rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t 
     if ((tid & 31) == 0) mbar_arrive(empty + slot);
 
     if constexpr (G == 1024)
-      transform_chunk<G>(v, xbuf, tt, perm << 1);
+      transform_chunk_1024_sa(v, xbuf_sa, tt, perm << 1);
     else
       transform_slots<G>(v);
     const unsigned m = __reduce_max_sync(row_lanes, __float_as_uint(chunk_absmax(v)));
@@ -398,7 +487,7 @@ inline bool ring_plan(int64_t M, int64_t K, int64_t K_pad, RingPlan& pl, size_t&
   pl.groups = (M + TR - 1) / TR;
   const size_t xbuf = (G == 1024) ? static_cast<size_t>(pl.teams) * pl.team_warps * 32 * 256 : 0;
   const size_t amax = (static_cast<size_t>(pl.teams) * 3 * TR + 1) / 2 * 8;
-  const size_t fixed = xbuf + amax + 16;
+  const size_t fixed = xbuf + amax + 16 + 1024;          // + alignment slack of the base
   if (fixed + pl.slot_bytes + 20 > static_cast<size_t>(kRingMaxSmem)) return false;
   // per slot: its bytes, two mbarriers and its claim word
   int slots = static_cast<int>((kRingMaxSmem - fixed) / (pl.slot_bytes + 20));
