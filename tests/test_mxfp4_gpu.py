@@ -117,6 +117,34 @@ def test_quant_mxfp4_matches_oracle(cuda_lib, g, M, K):
     assert cuda_lib.device_status() == 0
 
 
+GUARD = 0xA5
+
+
+@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("M,K", [(37, 3000), (130, 1088), (225, 1024)])
+def test_quant_mxfp4_writes_nothing_outside_its_outputs(cuda_lib, g, M, K):
+    """Guard bytes around every output: code rows wider than K4 / 2 and one guard row after the
+    last; the scale buffer longer than its layout, with the bytes the layout leaves unused
+    (padding atoms, weight-image lanes past the tile) filled too. Each must stay untouched."""
+    X = make_matrix(M, K, seed=M + K + 3 * g, std=1.0, row_outliers=3, row_scale=40.0)
+    K4 = cuda_lib.nvfp4_k(K, g)
+    for weights, tile_rows in ((False, TILE_A), (True, TILE_B)):
+        ldq = -(-(K4 // 2 + 32) // 16) * 16
+        q = torch.full((M + 1, ldq), GUARD, dtype=torch.uint8, device="cuda")
+        size = cuda_lib.mxfp4_scale_bytes(M, K, g, weights)
+        assert size == sf_size(M, K4 // 32, tile_rows)
+        sf = torch.full((size + 256,), GUARD, dtype=torch.uint8, device="cuda")
+        fn = cuda_lib.prepack_weight_mxfp4 if weights else cuda_lib.rotate_quant_act_mxfp4
+        fn(padded_rows(X), g, q=q[:M], sf=sf)
+        torch.cuda.synchronize()
+        what = f"{'wgt' if weights else 'act'} g{g} M{M} K{K}"
+        assert (q[:M, K4 // 2:] == GUARD).all() and (q[M] == GUARD).all(), what
+        used = np.zeros(size + 256, dtype=bool)
+        used[sf_index(M, K4 // 32, tile_rows).ravel()] = True
+        assert (sf.cpu().numpy()[~used] == GUARD).all(), f"{what}: scale bytes written outside the layout"
+        check_mx(q[:M], sf, X, g, tile_rows, what)
+
+
 def test_quant_mxfp4_zero_onehot_and_tiny_rows(cuda_lib):
     M, K, g = 8, 256, 64
     X = torch.zeros(M, K, dtype=torch.bfloat16)

@@ -127,6 +127,37 @@ def test_quant_nvfp4_matches_oracle(cuda_lib, g, M, K):
     check_fp4(qw, sfw, gw, X, g, TILE_B, f"wgt g{g} M{M} K{K}")
 
 
+GUARD = 0xA5
+
+
+@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("M,K", [(37, 3000), (130, 1088), (225, 1024)])
+def test_quant_nvfp4_writes_nothing_outside_its_outputs(cuda_lib, g, M, K):
+    """Guard bytes around every output: code rows wider than K4 / 2 and one guard row after the
+    last; the block-scale buffer longer than its layout, with the bytes the layout leaves unused
+    (an activation tile's padding atom when its chunk count is odd, weight-image lanes of rows
+    past the tile) filled too; guard row scales after row M - 1. Each must stay untouched."""
+    X = make_matrix(M, K, seed=M + K + g, std=1.0, row_outliers=3, row_scale=40.0)
+    K4 = cuda_lib.nvfp4_k(K, g)
+    for weights, tile_rows in ((False, TILE_A), (True, TILE_B)):
+        ldq = -(-(K4 // 2 + 32) // 16) * 16
+        q = torch.full((M + 1, ldq), GUARD, dtype=torch.uint8, device="cuda")
+        size = cuda_lib.nvfp4_scale_bytes(M, K, g, weights)
+        assert size == sf_size(M, K4 // 16, tile_rows)
+        sf = torch.full((size + 256,), GUARD, dtype=torch.uint8, device="cuda")
+        gs = torch.full((M + 8,), -123.0, dtype=torch.float32, device="cuda")
+        fn = cuda_lib.prepack_weight_nvfp4 if weights else cuda_lib.rotate_quant_act_nvfp4
+        fn(padded_rows(X), g, q=q[:M], sf=sf, g=gs[:M])
+        torch.cuda.synchronize()
+        what = f"{'wgt' if weights else 'act'} g{g} M{M} K{K}"
+        assert (q[:M, K4 // 2:] == GUARD).all() and (q[M] == GUARD).all(), what
+        assert (gs[M:] == -123.0).all(), what
+        used = np.zeros(size + 256, dtype=bool)
+        used[sf_index(M, K4 // 16, tile_rows).ravel()] = True
+        assert (sf.cpu().numpy()[~used] == GUARD).all(), f"{what}: scale bytes written outside the layout"
+        check_fp4(q[:M], sf, gs[:M], X, g, tile_rows, what)
+
+
 def test_quant_nvfp4_zero_and_onehot_rows(cuda_lib):
     M, K, g = 8, 256, 64
     X = torch.zeros(M, K, dtype=torch.bfloat16)
