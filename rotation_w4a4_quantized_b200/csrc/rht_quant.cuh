@@ -920,14 +920,15 @@ cudaError_t launch_reg_t(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, i
 // fit it.
 template <int G, int QM>
 cudaError_t launch_ring(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
-                        uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream);
+                        uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream, Fp4Out fp4);
 
 template <int G, int QM>
 cudaError_t launch_g(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
                      uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream) {
   // K a multiple of 8 and rows of at most 16384 columns: whole rows stream into a shared ring
   {
-    const cudaError_t e = launch_ring<G, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream);
+    const cudaError_t e = launch_ring<G, QM>(X, M, K, ldx, K_pad, Q, ldq, S, stream,
+                                             Fp4Out{nullptr, 0, 0, 0});
     if (e != cudaErrorNotSupported) return e;
   }
   // rows of up to 16384 columns: CTAs of at most 256 threads, two per SM; longer rows (at most
@@ -971,6 +972,11 @@ inline cudaError_t launch_rht_quant_fp4(const uint16_t* X, int64_t M, int64_t K,
   const quant_detail::Fp4Out o{sf, tile_rows, static_cast<int>(K4 / 64), layout};
 #define CONVROT_FP4_CASE(G)                                                                   \
   case G:                                                                                     \
+    if (G >= 256) {                                                                           \
+      const cudaError_t e = quant_detail::launch_ring<G, kQmFp4>(X, M, K, ldx, K4, Q, ldq, S, \
+                                                                 stream, o);                  \
+      if (e != cudaErrorNotSupported) return e;                                               \
+    }                                                                                         \
     return K4 <= 256 * quant_detail::kChunk                                                   \
                ? quant_detail::launch_reg_t<G, kQmFp4, 256, 2>(X, M, K, ldx, K4, Q, ldq, S,   \
                                                                stream, o)                     \

@@ -300,10 +300,17 @@ __device__ __forceinline__ void store_slots_small(const float (&v)[kChunk], floa
   }
 }
 
+// QM: 7 (packed int4), 127 (int8) or kQmFp4 (NVFP4, for G = 256 and 1024, whose register
+// layouts match the register kernel's, with K_pad = K4). MXFP4 stays on the register kernel,
+// which ran it faster (qkv 9.97 against 10.53 us here).
 template <int G, int QM>
 __global__ void __launch_bounds__(32 * (kRingMaxWarps + 1), 1)
 rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t ldx, int K_pad,
-                      uint8_t* __restrict__ Q, int64_t ldq, float* __restrict__ S, RingPlan pl) {
+                      uint8_t* __restrict__ Q, int64_t ldq, float* __restrict__ S, RingPlan pl,
+                      Fp4Out fp4) {
+  constexpr bool kFp = (QM == kQmFp4);
+  static_assert(QM != kQmMx, "MXFP4 runs on the register kernel");
+  static_assert(!kFp || G >= 256, "NVFP4: G = 256 or 1024 (slot layouts)");
   extern __shared__ __align__(1024) unsigned char smem_raw_rows[];
   // 1024-byte aligned base (the plan reserves the slack)
   unsigned char* smem_rows = smem_raw_rows + ((1024u - (smem_u32(smem_raw_rows) & 1023u)) & 1023u);
@@ -421,7 +428,20 @@ rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t 
       transform_chunk_1024_sa(v, xbuf_sa, tt, perm << 1);
     else
       transform_slots<G>(v);
-    const unsigned m = __reduce_max_sync(row_lanes, __float_as_uint(chunk_absmax(v)));
+    // NVFP4: the maxima of the four 16-column blocks (G = 1024 first regroups whole blocks per
+    // thread through the same exchange rows)
+    float bm[4];
+    float mx;
+    if constexpr (kFp) {
+      if constexpr (G == 1024)
+        blocks_1024(v, reinterpret_cast<float4*>(smem_rows) + 16 * team * team_threads, tt);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) bm[r] = absmax16(v + 16 * r);
+      mx = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3]));
+    } else {
+      mx = chunk_absmax(v);
+    }
+    const unsigned m = __reduce_max_sync(row_lanes, __float_as_uint(mx));
     const int64_t row = (g_begin + k) * pl.TR + r_local;
     const bool active = lane_ok && row < M;
     unsigned int* am = am_team + a3 * pl.TR;
@@ -430,7 +450,15 @@ rht_quant_ring_kernel(const uint16_t* __restrict__ X, int64_t M, int K, int64_t 
     if (team_barrier_or(bar_id, team_threads, !ok)) break;
     // the absmax slot of the previous round is no longer read by anyone: clear it for reuse
     if (tt < pl.TR) am_team[(a3 == 0 ? 2 : a3 - 1) * pl.TR + tt] = 0u;
-    if (active) {
+    if constexpr (QM == kQmFp4) {
+      float gr = 0.f;
+      if (active) {
+        constexpr float kNorm = 1.0f / static_cast<float>(1 << log4_of<G>());
+        gr = __fdiv_rn(__uint_as_float(am[r_local]) * kNorm, 6.0f * 448.0f);
+        if (c == 0) S[row] = gr;
+      }
+      store_fp4<G>(v, bm, gr, Q + (active ? row : 0) * ldq, row, c, j, fp4, active);
+    } else if (active) {
       float scale, inv;
       row_scale_fast<G, QM>(am[r_local], scale, inv);
       if (c == 0) S[row] = scale;
@@ -500,20 +528,25 @@ inline bool ring_plan(int64_t M, int64_t K, int64_t K_pad, RingPlan& pl, size_t&
 // Returns cudaErrorNotSupported when the shape does not fit the ring kernel.
 template <int G, int QM>
 cudaError_t launch_ring(const uint16_t* X, int64_t M, int64_t K, int64_t ldx, int64_t K_pad,
-                        uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream) {
-  RingPlan pl;
-  size_t smem = 0;
-  if (!ring_plan<G>(M, K, K_pad, pl, smem)) return cudaErrorNotSupported;
-  auto kern = rht_quant_ring_kernel<G, QM>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int64_t sms = sm_count();
-  const int64_t grid = pl.groups < sms ? pl.groups : sms;
-  const int threads = 32 * (1 + pl.teams * pl.team_warps);
-  return launch_overlapped(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
-                           X, M, static_cast<int>(K), ldx, static_cast<int>(K_pad), Q, ldq, S,
-                           pl);
+                        uint8_t* Q, int64_t ldq, float* S, cudaStream_t stream,
+                        Fp4Out fp4) {
+  if constexpr (QM == kQmMx || (QM == kQmFp4 && G < 256)) {
+    return cudaErrorNotSupported;   // MXFP4 and G <= 64 NVFP4: the register kernel
+  } else {
+    RingPlan pl;
+    size_t smem = 0;
+    if (!ring_plan<G>(M, K, K_pad, pl, smem)) return cudaErrorNotSupported;
+    auto kern = rht_quant_ring_kernel<G, QM>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int64_t sms = sm_count();
+    const int64_t grid = pl.groups < sms ? pl.groups : sms;
+    const int threads = 32 * (1 + pl.teams * pl.team_warps);
+    return launch_overlapped(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem,
+                             stream, X, M, static_cast<int>(K), ldx, static_cast<int>(K_pad), Q,
+                             ldq, S, pl, fp4);
+  }
 }
 
 }  // namespace quant_detail
