@@ -99,7 +99,7 @@ def l2_bytes(dev) -> int:
 
 KERNEL_SOURCES = ("capi.cu", "internal.h", "ptx.cuh", "rht_quant.cuh", "rht_quant_ring.cuh",
                   "gemm_common.cuh",
-                  "w4a4_gemm.cuh", "w8a8_gemm.cuh", "nvfp4_gemm.cuh")
+                  "w4a4_gemm.cuh", "w8a8_gemm.cuh", "nvfp4_gemm.cuh", "mxfp4_gemm.cuh")
 
 
 def kernel_sources_sha256():
@@ -114,9 +114,7 @@ def kernel_sources_sha256():
 def traffic_key(kernel_name: str):
     """The key a bench line uses for a kernel in ncu's report (None: not one of ours)."""
     import re
-    if re.search(r"nvfp4_gemm_kernel<[^,>]*,\s*(1|true)\s*>", kernel_name):   # <mode, kMx>
-        return "mxfp4_gemm_kernel"
-    for k in ("w4a4_gemm_kernel", "w8a8_gemm_kernel", "nvfp4_gemm_kernel"):
+    for k in ("w4a4_gemm_kernel", "w8a8_gemm_kernel", "nvfp4_gemm_kernel", "mxfp4_gemm_kernel"):
         if k in kernel_name:
             return k
     m = (re.search(r"rht_quant_reg_kernel<\s*\d+,\s*(\d+)", kernel_name)       # <G, QM, ...>

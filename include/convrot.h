@@ -179,8 +179,8 @@ int convrot_w8a8_gemm_s32(const uint8_t* qx, int64_t ldqx, const uint8_t* qw, in
  * group and 64-K chunk, the scale of row r and block b (of the 4 in the chunk) belongs at byte
  * 16 (r % 32) + 4 ((r % 128) / 32) + b of a 512-byte atom. Activations: rows in tiles of 128,
  * one atom per tile and chunk, the chunk count per tile rounded up to even (the padding atom is
- * not written). Weights: rows in tiles of 224 (the GEMM's N tile), one 4096-byte image per tile
- * and chunk: 128 lanes L x 32 bytes, lane L byte j at 256 (L / 8) + 128 (j / 16) + 16 (L % 8) +
+ * not written). Weights: rows in tiles of 192 (the NVFP4 GEMM's N tile), one 4096-byte image
+ * per tile and chunk: 128 lanes L x 32 bytes, lane L byte j at 256 (L / 8) + 128 (j / 16) + 16 (L % 8) +
  * j % 16, row r's scales in the four lanes L = r % 32 + 32 q (q = 0..3) at byte
  * 4 ((r % 128) / 32) + b of the half j / 16 = r / 128.
  * Buffer sizes come from convrot_nvfp4_scale_bytes. */
@@ -232,7 +232,7 @@ int convrot_nvfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
  * 128-K chunk, the scale of row r and block b (of the 4 in the chunk) belongs at byte
  * 16 (r % 32) + 4 ((r % 128) / 32) + b of a 512-byte atom; activations store the atoms (128-row
  * tiles, chunk count per tile rounded up to even), weights the 4-fold replicated 4096-byte
- * images of 224-row tiles. Buffer sizes come from convrot_mxfp4_scale_bytes; K4 from
+ * images of 224-row tiles (the MXFP4 GEMM's N tile). Buffer sizes come from convrot_mxfp4_scale_bytes; K4 from
  * convrot_nvfp4_k. */
 
 /* Bytes of the scale buffer for `rows` rows: operand 0 = activations, 1 = weights; -1 on bad

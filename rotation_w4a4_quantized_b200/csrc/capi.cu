@@ -15,6 +15,7 @@
 #include "rht_quant_ring.cuh"
 #include "w4a4_gemm.cuh"
 #include "w8a8_gemm.cuh"
+#include "mxfp4_gemm.cuh"
 #include "nvfp4_gemm.cuh"
 
 // Scratch of convrot_w4a4_linear_fused_noalloc (the packed activation codes and row scales of
@@ -379,24 +380,24 @@ int convrot_nvfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
 
 int64_t convrot_mxfp4_scale_bytes(int64_t rows, int64_t K, int group, int operand) {
   if (!valid_group(group) || K < 0 || rows < 0 || (operand != 0 && operand != 1)) return -1;
-  constexpr int kSfK = fp4_detail::kSfK<true>;
-  return operand == 0 ? nvfp4_sf_bytes(rows, nvfp4_k(K, group), fp4_detail::kSfTileA,
+  constexpr int kSfK = mx_detail::kSfK;
+  return operand == 0 ? nvfp4_sf_bytes(rows, nvfp4_k(K, group), mx_detail::kSfTileA,
                                        kSfActAtoms, kSfK)
-                      : nvfp4_sf_bytes(rows, nvfp4_k(K, group), fp4_detail::kSfTileB,
+                      : nvfp4_sf_bytes(rows, nvfp4_k(K, group), mx_detail::kSfTileB,
                                        kSfWeightImage, kSfK);
 }
 
 int convrot_rotate_quant_act_mxfp4(const uint16_t* X, int64_t M, int64_t K, int64_t ldx,
                                    int group, uint8_t* qx, int64_t ldq, uint8_t* sfx,
                                    convrot_stream_t stream) {
-  return rotate_quant_mx(X, M, K, ldx, group, qx, ldq, sfx, fp4_detail::kSfTileA, kSfActAtoms,
+  return rotate_quant_mx(X, M, K, ldx, group, qx, ldq, sfx, mx_detail::kSfTileA, kSfActAtoms,
                          stream);
 }
 
 int convrot_prepack_weight_mxfp4(const uint16_t* W, int64_t N, int64_t K, int64_t ldw, int group,
                                  uint8_t* qw, int64_t ldqw, uint8_t* sfw,
                                  convrot_stream_t stream) {
-  return rotate_quant_mx(W, N, K, ldw, group, qw, ldqw, sfw, fp4_detail::kSfTileB, kSfWeightImage,
+  return rotate_quant_mx(W, N, K, ldw, group, qw, ldqw, sfw, mx_detail::kSfTileB, kSfWeightImage,
                          stream);
 }
 
@@ -408,9 +409,9 @@ int convrot_mxfp4_linear(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, co
   if (st != CONVROT_OK || M == 0 || N == 0) return st;
   if (!aligned(bias, 2) || !aligned(Y, 2)) return CONVROT_ERR_ALIGN;
   if ((st = check_device()) != CONVROT_OK) return st;
-  return from_cuda(launch_nvfp4_gemm(qx, ldqx, sfx, nullptr, qw, ldqw, sfw, nullptr, bias, Y, ldy,
-                                     M, N, K4, GemmOut::kDequantBf16,
-                                     reinterpret_cast<cudaStream_t>(stream), true));
+  return from_cuda(launch_mxfp4_gemm(qx, ldqx, sfx, qw, ldqw, sfw, bias, Y, ldy, M, N, K4,
+                                     GemmOut::kDequantBf16,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int convrot_mxfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, const uint8_t* qw,
@@ -420,9 +421,8 @@ int convrot_mxfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
   if (st != CONVROT_OK || M == 0 || N == 0) return st;
   if (!aligned(acc, 4)) return CONVROT_ERR_ALIGN;
   if ((st = check_device()) != CONVROT_OK) return st;
-  return from_cuda(launch_nvfp4_gemm(qx, ldqx, sfx, nullptr, qw, ldqw, sfw, nullptr, nullptr, acc,
-                                     ldacc, M, N, K4, GemmOut::kRawS32,
-                                     reinterpret_cast<cudaStream_t>(stream), true));
+  return from_cuda(launch_mxfp4_gemm(qx, ldqx, sfx, qw, ldqw, sfw, nullptr, acc, ldacc, M, N, K4,
+                                     GemmOut::kRawS32, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int64_t convrot_w4a4_fused_workspace_bytes(int64_t M, int64_t K, int group) {

@@ -17,9 +17,11 @@ constexpr int64_t kMaxQuantKPad = 32768;
 constexpr int64_t kMaxGemmKPad = 131072;
 
 // NVFP4 block-scale layouts written by the quantisation and read by the block-scaled GEMM:
-// weights as 4096-byte images that one 128-lane tensor-memory copy reads (one per 224-row tile
-// and 64-K chunk); activations as 512-byte atoms (one per 128-row tile and 64-K chunk, the chunk
-// count per tile rounded up to even), which the GEMM's tensor copies expand into such images.
+// weights as 4096-byte images that one 128-lane tensor-memory copy reads (one per N tile of the
+// GEMM, 192 rows for NVFP4 and 224 for MXFP4, and chunk); activations as 512-byte atoms (one per
+// 128-row tile and chunk, the chunk count per tile rounded up to even). The MXFP4 GEMM's tensor
+// copies expand the atoms into such images; the NVFP4 GEMM reads the atoms and the first
+// quadrant of each weight image and writes the scales into tensor memory from its warps.
 enum Fp4SfLayout : int { kSfWeightImage = 0, kSfActAtoms = 1 };
 
 // Programmatic dependent launch: the hot kernels are launched with programmatic stream

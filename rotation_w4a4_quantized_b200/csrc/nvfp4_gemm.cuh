@@ -14,18 +14,22 @@
 // tiles (224 accumulator columns x 2 buffers + one stage of scale factors fill the 512 TMEM
 // columns). Per K stage (256 elements = 128 bytes per row) each CTA loads its 128 A rows, its
 // 112 B rows and the stage's block scales (A: its 128 rows; B: all 224 rows of the tile, the
-// same in both CTAs), pre-tiled in global memory in the order tcgen05.cp wants them; all copies
-// complete on the even CTA's barrier. The even CTA's MMA thread copies the scales into tensor
-// memory and issues 4 block-scaled MMAs (K = 64 each) per stage. One tcgen05.cp 128x256b (128
-// lanes x 8 columns) places the scales of two of A's 64-K chunks, or both 128-row halves of one
-// of B's, from a 4-fold replicated 4096-byte image: 2 + 4 copies per stage. B's images come
-// from the weight prepack; A's are assembled by the loads themselves: the activation
-// quantisation writes plain 512-byte atoms, and per pair of chunks four 1 KB tensor copies
-// (one per lane quadrant, a 5-D view of the atoms whose box interleaves the two chunks' 128-byte
-// pieces) build the image in shared memory. The copies run in the tensor pipe in issue order with the MMAs and
-// cost about as much as one MMA each, so fewer copies is the lever. One scale region serves
-// every stage. Epilogue as in the integer GEMMs (fp32 accumulator), one staging block per warp
-// (shared memory is short). Every wait is bounded.
+// same in both CTAs); the code tiles complete on the even CTA's barrier, the scales on a barrier
+// of their own CTA. The MMA reads a 64-K chunk's scales (4 per row) from 4 tensor-memory
+// columns of 32 lanes, the same in every lane quadrant (A: row r at lane r % 32, column r / 32;
+// B: two such groups of 4 columns, one per 128-row half of the tile). Four scale warps per CTA,
+// one per lane quadrant, write them there with tcgen05.st from the plain layouts in shared
+// memory (A: the 512-byte atoms the activation quantisation writes; B: the first lane quadrant,
+// 1 KB, of each 4096-byte weight image), so only the 6 KB of distinct scales per stage cross
+// from L2 (the replicated images were 24 KB, and the kernel is bound by the bytes it moves into
+// shared memory), and the tensor pipe runs no copies (a tcgen05.cp cost about as much as an
+// MMA). Scales go through two tensor-memory buffers: the warps fill buffer g % 2 with stage
+// g's scales once the MMAs of stage g - 2 have completed (the stage's own tcgen05.commit on
+// `empty`: a commit costs the tensor pipe about as much as an MMA, so there is one per stage),
+// while the MMAs of stage g - 1 run. The even
+// CTA's MMA thread issues 4 block-scaled MMAs (K = 64 each) per stage. Epilogue as in the
+// integer GEMMs (fp32 accumulator), one staging block per warp (shared memory is short).
+// Every wait is bounded.
 #pragma once
 
 #include <cuda.h>
@@ -46,20 +50,26 @@ using gemm_common::kEpiWarps;
 
 constexpr int BM = 256;          // tile rows per CTA pair
 constexpr int BMC = BM / 2;      // A rows per CTA (TMEM lanes)
-constexpr int BN = 224;          // tile columns (accumulator columns)
+constexpr int BN = 192;          // tile columns (accumulator columns)
 constexpr int BNC = BN / 2;      // B rows per CTA
 constexpr int BKB = 128;         // bytes of packed e2m1 per row per stage (256 K)
 constexpr int kChunks = 4;       // MMAs (64 K each) per stage
 #ifndef CONVROT_FP4_STAGES
-#define CONVROT_FP4_STAGES 4
+#define CONVROT_FP4_STAGES 6
 #endif
 constexpr int SU = CONVROT_FP4_STAGES;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kSfWarps = 4;      // scale warps (one per TMEM lane quadrant)
+constexpr int kThreads = 32 * (2 + kEpiWarps + kSfWarps);
 constexpr int kAccCols = BN;
 constexpr int kTmemCols = 512;
-constexpr int kSfaCol = 2 * kAccCols;                  // 448: 4 columns per chunk
-constexpr int kSfbCol = kSfaCol + 4 * kChunks;         // 464: 8 columns per chunk
-static_assert(kSfbCol + 8 * kChunks <= kTmemCols, "TMEM budget");
+// two scale buffers (stage g in buffer g % 2), each A (4 columns per chunk) then B (8 columns
+// per chunk)
+constexpr int kSfCol = 2 * kAccCols;                   // 384
+constexpr int kSfBufCols = 12 * kChunks;               // 48
+constexpr int kSfbOff = 4 * kChunks;                   // 16
+static_assert(kSfCol % 8 == 0 && kSfBufCols % 8 == 0 && kSfbOff % 8 == 0 &&
+                  kSfCol + 2 * kSfBufCols <= kTmemCols,
+              "TMEM budget");
 
 // tile rows of the block-scale layouts (activations: 128-row tiles of atoms; weights: 224-row
 // tiles of images)
@@ -70,16 +80,13 @@ constexpr int kEpiSmem = kEpiWarps * kEpiBufs * gemm_common::kStageBytes;
 
 constexpr int kTA = BMC * BKB;               // 16 KB
 constexpr int kTB = BNC * BKB;               // 14 KB
-// Scale chunks (4 scales per row each) cover 64 K (NVFP4, one scale per 16) or 128 K (MXFP4,
-// one per 32): 4 or 2 per stage. Shared memory is laid out for the larger NVFP4 stage.
-template <bool kMx> constexpr int kSfK = kMx ? 128 : 64;
-template <bool kMx> constexpr int kSfChunks = BKB * 2 / kSfK<kMx>;          // per stage
-template <bool kMx> constexpr int kSAt = kSfChunks<kMx> / 2 * 4096;        // A pair images
-template <bool kMx> constexpr int kSBt = kSfChunks<kMx> * 4096;            // B images
-template <bool kMx>
-constexpr uint32_t kStageTx = 2u * (kTA + kTB + kSAt<kMx> + kSBt<kMx>);
-constexpr int kSA = kSAt<false>;             // 8 KB of A scales per stage (NVFP4)
-constexpr int kSB = kSBt<false>;             // 16 KB of B scales per stage (128 lanes x 32 B)
+// Scale chunks hold 4 scales per row and cover 64 K: 4 per stage.
+constexpr int kSfK = 64;
+constexpr int kSfChunks = BKB * 2 / kSfK;                // per stage
+constexpr int kSA = kSfChunks * 512;                     // 2 KB: A's atoms of a stage
+constexpr int kSB = kSfChunks * 1024;                    // 4 KB: B images' first quadrants
+constexpr uint32_t kStageTx = 2u * (kTA + kTB);          // code tiles of the pair
+constexpr uint32_t kSfTx = kSA + kSB;                    // this CTA's scales
 
 struct Smem {
   static constexpr int uA = 0;
@@ -88,7 +95,7 @@ struct Smem {
   static constexpr int sB = sA + SU * kSA;
   static constexpr int stg = sB + SU * kSB;
   static constexpr int bars = stg + kEpiSmem;
-  static constexpr int n_bars = 2 * SU + 4 + 1;
+  static constexpr int n_bars = 3 * SU + 4 + 1 + 2;
   static constexpr int misc = bars + n_bars * 8;
   static constexpr int total = misc + 16;
 };
@@ -98,7 +105,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 using TileGrid = gemm_common::TileGrid<BM, BN>;
 
-template <GemmOut kMode, bool kMx>
+template <GemmOut kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -114,6 +121,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint64_t* acc_full = bars + 2 * SU;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
+  uint64_t* sf_full = mma_done + 1;          // this CTA's scales of a stage have landed
+  uint64_t* sf_ready = sf_full + SU;         // (even CTA) a scale buffer is written in both CTAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + Smem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + Smem::misc + 4);
 
@@ -126,14 +135,15 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int num_tiles = grid.count();
   const int kc_total = K4 / 64;                          // 64-K chunks per row
   const int num_k = (kc_total + kChunks - 1) / kChunks;  // stages per tile
-  constexpr int kMmaPerSf = kSfK<kMx> / 64;              // MMAs per scale chunk
-  const int sf_total = (K4 + kSfK<kMx> - 1) / kSfK<kMx>; // scale chunks per row
+  const int sf_total = (K4 + kSfK - 1) / kSfK;           // scale chunks per row
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SU; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
+      mbar_init(sf_full + i, 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(sf_ready + i, 2 * kSfWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 2 * kEpiWarps);
@@ -177,22 +187,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(full + slot, kStageTx<kMx>);
+          if (rank == 0) mbar_arrive_expect_tx(full + slot, kStageTx);
           const uint32_t bar = full_even + slot * 8;
           tma_load_2d_pair(base + Smem::uA + slot * kTA, &tmA, bar, s * BKB,
                            m0 + static_cast<int>(rank) * BMC);
           tma_load_2d_pair(base + Smem::uB + slot * kTB, &tmB, bar, s * BKB,
                            n0 + static_cast<int>(rank) * BNC);
-          // A: per pair of chunks, one 1 KB copy of the two atoms into each lane quadrant
-          // of the pair's image (box {128 B, 2 chunks, 4 pieces}); pairs past the tile's
-          // end read zeros
-          for (int p = 0; p < kSfChunks<kMx> / 2; ++p)
-            for (int q = 0; q < 4; ++q)
-              tma_load_5d_pair(base + Smem::sA + slot * kSA + p * 4096 + q * 1024, &tmSA, bar,
-                               0, 0, 0, s * (kSfChunks<kMx> / 2) + p, a_tile);
-          // B: images viewed as rows of 128 bytes (32 per image), one per scale chunk
-          tma_load_2d_pair(base + Smem::sB + slot * kSB, &tmSB, bar, 0,
-                           (b_tile * sf_total + s * kSfChunks<kMx>) * 32);
+          // this CTA's scales: A's atoms of the stage (rows of 128 bytes, 4 per atom; atoms
+          // past the tile's end read zeros) and the first 8 of each B image's 32 rows
+          mbar_arrive_expect_tx(sf_full + slot, kSfTx);
+          tma_load_3d(base + Smem::sA + slot * kSA, &tmSA, sf_full + slot, 0,
+                      s * kSfChunks * 4, a_tile);
+          tma_load_3d(base + Smem::sB + slot * kSB, &tmSB, sf_full + slot, 0, 0,
+                      b_tile * sf_total + s * kSfChunks);
         }
       }
       if (rank == 0) {
@@ -206,9 +213,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_fp4_bs(BM, BN, kMx);
-      const uint32_t sfa = tmem_base + kSfaCol;
-      const uint32_t sfb = tmem_base + kSfbCol;
+      constexpr uint32_t idesc = idesc_fp4_bs(BM, BN);
       uint32_t g = 0;
       int ti = 0;
       bool ok = true;
@@ -217,7 +222,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         if (ti >= 2 && !mbar_wait_cluster(acc_empty + b, ((ti >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * kAccCols;
-        for (int s = 0; s < num_k; ++s, ++g) {
+        for (int s = 0; s < num_k && ok; ++s, ++g) {
           const uint32_t slot = g % SU;
           if (!mbar_wait_cluster(full + slot, (g / SU) & 1, abort_flag)) {
             ok = false;
@@ -227,23 +232,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           const int nck = (kc_total - s * kChunks) < kChunks ? (kc_total - s * kChunks) : kChunks;
           const uint32_t a0 = smem_u32(base + Smem::uA + slot * kTA);
           const uint32_t b0 = smem_u32(base + Smem::uB + slot * kTB);
-          const uint32_t sa0 = smem_u32(base + Smem::sA + slot * kSA);
-          const uint32_t sb0 = smem_u32(base + Smem::sB + slot * kSB);
-          const int nsf = (nck + kMmaPerSf - 1) / kMmaPerSf;   // scale chunks in this stage
-          for (int p = 0; 2 * p < nsf; ++p)
-            tmem_cp_128x256b_pair(sfa + 8 * p, smem_desc_rows32(sa0 + 4096 * p));
-          for (int q = 0; q < nsf; ++q)
-            tmem_cp_128x256b_pair(sfb + 8 * q, smem_desc_rows32(sb0 + 4096 * q));
+          // CTA-scope acquire: the writers' tcgen05.wait::st completed their stores before
+          // they arrived
+          if (!mbar_wait(sf_ready + (g & 1), (g >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa = tmem_base + kSfCol + (g & 1) * kSfBufCols;
+          const uint32_t sfb = sfa + kSfbOff;
           for (int q = 0; q < nck; ++q) {
-            const int sc = q / kMmaPerSf;                     // this MMA's scale chunk
             const uint32_t acc = (s > 0 || q > 0) ? 1u : 0u;
-            if constexpr (kMx)
-              mma_mxf4_bs_pair(d_tmem, smem_desc_k128(a0 + q * 32), smem_desc_k128(b0 + q * 32),
-                               idesc_sf_ids(idesc, 2u * (q & 1)), sfa + 4 * sc, sfb + 8 * sc,
-                               acc);
-            else
-              mma_fp4_bs_pair(d_tmem, smem_desc_k128(a0 + q * 32), smem_desc_k128(b0 + q * 32),
-                              idesc, sfa + 4 * sc, sfb + 8 * sc, acc);
+            mma_fp4_bs_pair(d_tmem, smem_desc_k128(a0 + q * 32), smem_desc_k128(b0 + q * 32),
+                            idesc, sfa + 4 * q, sfb + 8 * q, acc);
           }
           mma_commit_pair(empty + slot, 0x3);
         }
@@ -256,7 +257,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       while (!mbar_try_wait_cluster(mma_done, 0) && ++polls < kMaxPolls) {
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;
     const uint32_t acc_empty_even = mapa_shared(smem_u32(acc_empty), 0);
@@ -271,11 +272,58 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       grid.coords(t, m0, n0);
       const int row0 = m0 + static_cast<int>(rank) * BMC + q * 32;
       const uint32_t acc_tmem = tmem_base + b * kAccCols + (static_cast<uint32_t>(q * 32) << 16);
-      gemm_common::epilogue_tile<kMode, BN, 0, true, kEpiBufs, !kMx>(
+      gemm_common::epilogue_tile<kMode, BN, 0, true, kEpiBufs, true>(
           acc_tmem, row0, n0, M, N, gx, gw, bias, out, ldo, tma_out, &tmY, stg, nstore,
           acc_empty_even + b * 8);
     }
     if (lane == 0) bulk_wait_group<0>();
+  } else {
+    // ------------------------------------------------------------------ scale warps (6..9)
+    // Warp w writes TMEM lanes 32 (w % 4) .. + 31; each lane L holds row L of every scale
+    // group: A's atom bytes 16 L .. 16 L + 15 (4 columns), B's half h at 256 (L / 8) + 128 h +
+    // 16 (L % 8) of the image's first quadrant (4 columns per half).
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t ready_even = mapa_shared(smem_u32(sf_ready), 0);
+    const uint32_t b_off = 256u * static_cast<uint32_t>(lane >> 3) + 16u * (lane & 7);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+      for (int s = 0; s < num_k; ++s, ++g) {
+        const uint32_t slot = g % SU;
+        ok = __all_sync(0xffffffffu, mbar_wait(sf_full + slot, (g / SU) & 1, abort_flag));
+        if (!ok) break;
+        // the stage's scales into registers (whole staging area; chunks past the tile's end
+        // land in columns no MMA reads), then into buffer g % 2 with one store per operand
+        constexpr int kC = kSfChunks;
+        const unsigned char* sa = base + Smem::sA + slot * kSA + 16 * lane;
+        const unsigned char* sb = base + Smem::sB + slot * kSB + b_off;
+        uint32_t ra[4 * kC], rb[8 * kC];
+#pragma unroll
+        for (int k = 0; k < kC; ++k) {
+          const uint4 va = *reinterpret_cast<const uint4*>(sa + 512 * k);
+          const uint4 vb0 = *reinterpret_cast<const uint4*>(sb + 1024 * k);
+          const uint4 vb1 = *reinterpret_cast<const uint4*>(sb + 1024 * k + 128);
+          ra[4 * k] = va.x; ra[4 * k + 1] = va.y; ra[4 * k + 2] = va.z; ra[4 * k + 3] = va.w;
+          rb[8 * k] = vb0.x; rb[8 * k + 1] = vb0.y; rb[8 * k + 2] = vb0.z; rb[8 * k + 3] = vb0.w;
+          rb[8 * k + 4] = vb1.x; rb[8 * k + 5] = vb1.y; rb[8 * k + 6] = vb1.z;
+          rb[8 * k + 7] = vb1.w;
+        }
+        // buffer g % 2 was last read by the MMAs of stage g - 2 (their commit on `empty`)
+        if (g >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(empty + (g - 2) % SU, ((g - 2) / SU) & 1, abort_flag));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const uint32_t sfa = lane_base + kSfCol + (g & 1) * kSfBufCols;
+        tmem_st_32x32b_x16(sfa, ra);
+        tmem_st_32x32b_x32(sfa + kSfbOff, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ready_even + 8 * (g & 1));
+      }
+    }
   }
 
   tc_fence_before();
@@ -287,12 +335,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   }
 }
 
-template <GemmOut kMode, bool kMx>
+template <GemmOut kMode>
 cudaError_t launch_mode(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                         const CUtensorMap& tmSB, const CUtensorMap& tmY, const float* gx,
                         const float* gw, const uint16_t* bias, void* out, int64_t ldo, int64_t M,
                         int64_t N, int64_t K4, int tma_out, cudaStream_t stream) {
-  auto k = nvfp4_gemm_kernel<kMode, kMx>;
+  auto k = nvfp4_gemm_kernel<kMode>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -305,22 +353,36 @@ cudaError_t launch_mode(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
                            tma_out);
 }
 
-// The activation scale atoms as a 5-D tensor {128 bytes, chunk parity (2), 128-byte piece (4),
-// chunk pair, 128-row tile}: a {128, 2, 4, 1, 1} box lands in shared memory as one lane
-// quadrant of the pair's 4096-byte image (piece p of chunk 2k + h at 256 p + 128 h). A chunk
-// holds 4 scales per row: sf_k = 64 (NVFP4) or 128 (MXFP4) columns of K.
-inline bool make_act_scale_map(CUtensorMap* map, const uint8_t* sfx, int64_t M, int64_t K4,
-                               int sf_k) {
+// The activation scale atoms as a 3-D tensor {128 bytes, 128-byte row (4 per atom, chunk-major),
+// 128-row tile}: a {128, 4 x chunks per stage, 1} box is one stage's atoms. A chunk holds 4
+// scales per row (64 columns of K).
+inline bool make_act_scale_map(CUtensorMap* map, const uint8_t* sfx, int64_t M, int64_t K4) {
+  constexpr int sf_k = kSfK, chunks_per_stage = kSfChunks;
   auto enc = gemm_common::get_encode_fn();
   if (!enc) return false;
   const int64_t kc_even = ((K4 + sf_k - 1) / sf_k + 1) & ~int64_t(1);
   const int64_t tiles = (M + kSfTileA - 1) / kSfTileA;
-  cuuint64_t dims[5] = {128, 2, 4, static_cast<cuuint64_t>(kc_even / 2),
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(4 * kc_even),
                         static_cast<cuuint64_t>(tiles)};
-  cuuint64_t strides[4] = {512, 128, 1024, static_cast<cuuint64_t>(kc_even * 512)};
-  cuuint32_t box[5] = {128, 2, 4, 1, 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<uint8_t*>(sfx), dims, strides, box,
+  cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(kc_even * 512)};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(4 * chunks_per_stage), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(sfx), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The weight scale images as a 3-D tensor {128 bytes, 128-byte row (32 per image), image}: a
+// {128, 8, chunks per stage} box is the first lane quadrant of one stage's images.
+inline bool make_weight_scale_map(CUtensorMap* map, const uint8_t* sfw, int64_t images) {
+  constexpr int chunks_per_stage = kSfChunks;
+  auto enc = gemm_common::get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, 32, static_cast<cuuint64_t>(images)};
+  cuuint64_t strides[2] = {128, 4096};
+  cuuint32_t box[3] = {128, 8, static_cast<cuuint32_t>(chunks_per_stage)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(sfw), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -341,32 +403,23 @@ inline cudaError_t launch_nvfp4_gemm(const uint8_t* qx, int64_t ldqx, const uint
                                      const float* gx, const uint8_t* qw, int64_t ldqw,
                                      const uint8_t* sfw, const float* gw, const uint16_t* bias,
                                      void* out, int64_t ldo, int64_t M, int64_t N, int64_t K4,
-                                     GemmOut mode, cudaStream_t stream, bool mx = false) {
+                                     GemmOut mode, cudaStream_t stream) {
   using namespace fp4_detail;
-  const int sf_k = mx ? kSfK<true> : kSfK<false>;
   CUtensorMap tmA, tmB, tmSA, tmSB, tmY;
   std::memset(&tmY, 0, sizeof(tmY));
   if (!gemm_common::make_u8_map(&tmA, qx, M, K4 / 2, ldqx, BKB, BMC, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!gemm_common::make_u8_map(&tmB, qw, N, K4 / 2, ldqw, BKB, BNC, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // scale buffers viewed as rows of 128 bytes
-  const int64_t sb_rows = nvfp4_sf_bytes(N, K4, kSfTileB, kSfWeightImage, sf_k) / 128;
-  if (!make_act_scale_map(&tmSA, sfx, M, K4, sf_k)) return cudaErrorInvalidValue;
-  if (!gemm_common::make_u8_map(&tmSB, sfw, sb_rows, 128, 128, 128,
-                                (mx ? kSBt<true> : kSBt<false>) / 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
+  const int64_t images = nvfp4_sf_bytes(N, K4, kSfTileB, kSfWeightImage) / 4096;
+  if (!make_act_scale_map(&tmSA, sfx, M, K4)) return cudaErrorInvalidValue;
+  if (!make_weight_scale_map(&tmSB, sfw, images)) return cudaErrorInvalidValue;
   const int tma_out = gemm_common::setup_out_map(&tmY, mode, out, M, N, ldo);
   if (mode == GemmOut::kDequantBf16)
-    return mx ? launch_mode<GemmOut::kDequantBf16, true>(tmA, tmB, tmSA, tmSB, tmY, gx, gw, bias,
-                                                         out, ldo, M, N, K4, tma_out, stream)
-              : launch_mode<GemmOut::kDequantBf16, false>(tmA, tmB, tmSA, tmSB, tmY, gx, gw,
-                                                          bias, out, ldo, M, N, K4, tma_out,
-                                                          stream);
-  return mx ? launch_mode<GemmOut::kRawS32, true>(tmA, tmB, tmSA, tmSB, tmY, gx, gw, bias, out,
-                                                  ldo, M, N, K4, 0, stream)
-            : launch_mode<GemmOut::kRawS32, false>(tmA, tmB, tmSA, tmSB, tmY, gx, gw, bias, out,
-                                                   ldo, M, N, K4, 0, stream);
+    return launch_mode<GemmOut::kDequantBf16>(tmA, tmB, tmSA, tmSB, tmY, gx, gw, bias, out, ldo,
+                                              M, N, K4, tma_out, stream);
+  return launch_mode<GemmOut::kRawS32>(tmA, tmB, tmSA, tmSB, tmY, gx, gw, bias, out, ldo, M, N,
+                                       K4, 0, stream);
 }
 
 }  // namespace convrot

@@ -285,15 +285,16 @@ __device__ __forceinline__ void store_row_codes(const float (&v)[kChunk], float 
 // the chunk) belongs at byte 16 (r % 32) + 4 ((r % 128) / 32) + b of a 512-byte atom.
 //  * activations (tiles of 128 rows): the atoms themselves, one per tile and chunk, the chunk
 //    count per tile rounded up to even (the padding atom is never written);
-//  * weights (tiles of 224 rows, the GEMM's N tile): one 4096-byte image per tile and chunk, the
-//    layout one 128-lane copy reads: 128 lanes L of 32 bytes, lane L byte j at 256 (L / 8) +
-//    128 (j / 16) + 16 (L % 8) + j % 16; row r's scales are in the four lanes L = r % 32 + 32 q
-//    (q = 0..3) at byte 4 ((r % 128) / 32) + b of the half j / 16 = r / 128.
+//  * weights (tiles of the GEMM's N tile: 192 rows for NVFP4, 224 for MXFP4): one 4096-byte
+//    image per tile and chunk, the layout one 128-lane copy reads: 128 lanes L of 32 bytes,
+//    lane L byte j at 256 (L / 8) + 128 (j / 16) + 16 (L % 8) + j % 16; row r's scales are in
+//    the four lanes L = r % 32 + 32 q (q = 0..3) at byte 4 ((r % 128) / 32) + b of the half
+//    j / 16 = r / 128.
 constexpr int kQmFp4 = 6;
 
 struct Fp4Out {
   uint8_t* sf;        // block scales (as above)
-  int tile_rows;      // 224 (weights) or 128 (activations)
+  int tile_rows;      // 192 / 224 (NVFP4 / MXFP4 weights) or 128 (activations)
   int kc_per_row;     // chunks of 4 scales per row: K4 / 64 (NVFP4), ceil(K4 / 128) (MXFP4)
   int layout;         // Fp4SfLayout
 };

@@ -50,13 +50,13 @@ def test_traffic_key_names_every_reported_kernel():
     assert bench.traffic_key("void convrot::gemm_detail::w4a4_gemm_kernel<0>(...)") == "w4a4_gemm_kernel"
     assert bench.traffic_key("w8a8_gemm_kernel<0>") == "w8a8_gemm_kernel"
     assert bench.traffic_key("nvfp4_gemm_kernel<0>") == "nvfp4_gemm_kernel"
-    assert bench.traffic_key("void convrot::nvfp4_gemm_kernel<(GemmMode)0, false>(...)") \
+    assert bench.traffic_key("void convrot::fp4_detail::nvfp4_gemm_kernel<(GemmOut)0>(...)") \
         == "nvfp4_gemm_kernel"
-    assert bench.traffic_key("void convrot::nvfp4_gemm_kernel<(GemmMode)0, true>(...)") \
+    assert bench.traffic_key("void convrot::mx_detail::mxfp4_gemm_kernel<(GemmOut)0>(...)") \
         == "mxfp4_gemm_kernel"
     # the forms ncu prints
-    assert bench.traffic_key("void fp4_detail::nvfp4_gemm_kernel<0, 0>(CUtensorMap_st, ...)") \
+    assert bench.traffic_key("void fp4_detail::nvfp4_gemm_kernel<0>(CUtensorMap_st, ...)") \
         == "nvfp4_gemm_kernel"
-    assert bench.traffic_key("void fp4_detail::nvfp4_gemm_kernel<0, 1>(CUtensorMap_st, ...)") \
+    assert bench.traffic_key("void mx_detail::mxfp4_gemm_kernel<0>(CUtensorMap_st, ...)") \
         == "mxfp4_gemm_kernel"
     assert bench.traffic_key("rht_quant_reg_kernel<256, 5, 256, 2>") == "rht_quant_kernel_mx"

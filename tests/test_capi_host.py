@@ -132,7 +132,7 @@ def test_nvfp4_host_helpers_and_validation(b):
                 assert b.lib.convrot_nvfp4_scale_bytes(rows, K, g, 0) == \
                     -(-rows // 128) * ((K4 // 64 + 1) // 2 * 2) * 512   # atoms, even count
                 assert b.lib.convrot_nvfp4_scale_bytes(rows, K, g, 1) == \
-                    -(-rows // 224) * (K4 // 64) * 4096              # one image per chunk
+                    -(-rows // 192) * (K4 // 64) * 4096              # one image per chunk
     assert b.lib.convrot_nvfp4_k(10, 32) == -1 and b.lib.convrot_nvfp4_scale_bytes(4, 64, 16, 2) == -1
     q4 = b.lib.convrot_rotate_quant_act_nvfp4
     assert q4(FAKE, 4, 64, 64, 16, FAKE, 16, FAKE, FAKE, None) == 2      # ldq < K4 / 2

@@ -22,12 +22,12 @@ from tests.parity import (CODE_MATCH, SCALE_RTOL, Y_FROB, bf16_to_f64, check_sca
 pytestmark = pytest.mark.gpu
 
 GROUPS = (16, 64, 256, 1024)
-TILE_A, TILE_B = 128, 224
+TILE_A, TILE_B = 128, 192
 
 
 def sf_index(rows, nblk, tile_rows):
     """Byte offsets [rows, nblk, replicas] of block scale (r, b), as stated in
-    include/convrot.h: weights (224-row tiles) as 4096-byte images, one per 64-K chunk, in four
+    include/convrot.h: weights (192-row tiles) as 4096-byte images, one per 64-K chunk, in four
     replicas; activations (128-row tiles) as 512-byte atoms, the chunk count per tile rounded
     up to even, one replica."""
     r = np.arange(rows)[:, None, None]
@@ -69,7 +69,7 @@ def tile(sb_bytes: np.ndarray, tile_rows) -> torch.Tensor:
 def test_scale_layouts_are_injective(tile_rows, rows, nblk):
     """Host check of the test's own index map: no byte is used twice and every index is inside
     the buffer; whole activation tiles with an even chunk count fill it exactly (weights leave
-    lanes of rows past 224 unused; an odd chunk count leaves a padding atom per tile)."""
+    lanes of rows past 192 unused; an odd chunk count leaves a padding atom per tile)."""
     idx = sf_index(rows, nblk, tile_rows)
     size = sf_size(rows, nblk, tile_rows)
     assert len(np.unique(idx)) == idx.size and idx.max() < size
