@@ -232,8 +232,8 @@ int convrot_nvfp4_gemm_f32(const uint8_t* qx, int64_t ldqx, const uint8_t* sfx, 
  * 128-K chunk, the scale of row r and block b (of the 4 in the chunk) belongs at byte
  * 16 (r % 32) + 4 ((r % 128) / 32) + b of a 512-byte atom; activations store the atoms (128-row
  * tiles, chunk count per tile rounded up to even), weights the 4-fold replicated 4096-byte
- * images of 224-row tiles (the MXFP4 GEMM's N tile). Buffer sizes come from convrot_mxfp4_scale_bytes; K4 from
- * convrot_nvfp4_k. */
+ * images of 224-row tiles (the MXFP4 GEMM's N tile). Buffer sizes come from
+ * convrot_mxfp4_scale_bytes; K4 from convrot_nvfp4_k. */
 
 /* Bytes of the scale buffer for `rows` rows: operand 0 = activations, 1 = weights; -1 on bad
  * arguments. Pure host function. */
