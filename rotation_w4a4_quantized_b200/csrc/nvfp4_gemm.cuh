@@ -209,6 +209,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           }
         }
       }
+      // this CTA's scale loads complete on its own barrier; on a normal exit the scale warps
+      // have consumed every phase, after a wait that gave up some may still be landing: let
+      // them land before the CTA's shared memory goes away
+      for (uint32_t s = (g > SU ? g - SU : 0); s < g; ++s) {
+        uint32_t polls = 0;
+        while (!mbar_try_wait(sf_full + (s % SU), (s / SU) & 1) && ++polls < kMaxPolls) {
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
