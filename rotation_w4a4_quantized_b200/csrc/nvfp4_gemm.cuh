@@ -10,26 +10,21 @@
 //
 // How (B200 design): e2m1 is a native operand type of tcgen05.mma kind::mxf4nvf4, read packed
 // (two per byte) from shared memory, so the codes go from HBM to the tensor cores by TMA with no
-// conversion stage; the block scales ride along. Persistent CTA pairs walk 256 x 224 output
-// tiles (224 accumulator columns x 2 buffers + one stage of scale factors fill the 512 TMEM
-// columns). Per K stage (256 elements = 128 bytes per row) each CTA loads its 128 A rows, its
-// 112 B rows and the stage's block scales (A: its 128 rows; B: all 224 rows of the tile, the
-// same in both CTAs); the code tiles complete on the even CTA's barrier, the scales on a barrier
-// of their own CTA. The MMA reads a 64-K chunk's scales (4 per row) from 4 tensor-memory
-// columns of 32 lanes, the same in every lane quadrant (A: row r at lane r % 32, column r / 32;
-// B: two such groups of 4 columns, one per 128-row half of the tile). Four scale warps per CTA,
-// one per lane quadrant, write them there with tcgen05.st from the plain layouts in shared
-// memory (A: the 512-byte atoms the activation quantisation writes; B: the first lane quadrant,
-// 1 KB, of each 4096-byte weight image), so only the 6 KB of distinct scales per stage cross
-// from L2 (the replicated images were 24 KB, and the kernel is bound by the bytes it moves into
-// shared memory), and the tensor pipe runs no copies (a tcgen05.cp cost about as much as an
-// MMA). Scales go through two tensor-memory buffers: the warps fill buffer g % 2 with stage
-// g's scales once the MMAs of stage g - 2 have completed (the stage's own tcgen05.commit on
-// `empty`: a commit costs the tensor pipe about as much as an MMA, so there is one per stage),
-// while the MMAs of stage g - 1 run. The even
-// CTA's MMA thread issues 4 block-scaled MMAs (K = 64 each) per stage. Epilogue as in the
-// integer GEMMs (fp32 accumulator), one staging block per warp (shared memory is short).
-// Every wait is bounded.
+// conversion stage. Persistent CTA pairs walk 256 x 192 output tiles. Per K stage (256 elements
+// = 128 bytes per row) each CTA loads its 128 A rows and its 96 B rows (completing on the even
+// CTA's barrier) and the stage's distinct block-scale bytes (completing on its own barrier):
+// A's 512-byte atoms as the activation quantisation writes them, and the first lane quadrant
+// (1 KB) of each of B's 4096-byte weight images, 6 KB in all. The MMA reads a 64-K chunk's
+// scales (4 per row) from 4 tensor-memory columns of 32 lanes, the same in every lane quadrant
+// (A: row r at lane r % 32, column r / 32; B: two such groups of 4 columns, one per 128-row half
+// of the tile). Four scale warps per CTA, one per lane quadrant, put them there with
+// tcgen05.st, so the tensor pipe runs no tcgen05.cp (the copies run in order with the MMAs and
+// cost it about 30 ns each). Tensor memory holds two 192-column accumulators and two
+// 48-column scale buffers: the warps fill buffer g % 2 with stage g's scales once the MMAs of
+// stage g - 2 have completed (that stage's own commit on `empty`), while the MMAs of stage
+// g - 1 run. The even CTA's MMA thread waits for a stage's codes and scales and issues its 4
+// block-scaled MMAs (K = 64 each). Epilogue as in the integer GEMMs (fp32 accumulator), one
+// staging block per warp. Every wait is bounded.
 #pragma once
 
 #include <cuda.h>
@@ -71,7 +66,7 @@ static_assert(kSfCol % 8 == 0 && kSfBufCols % 8 == 0 && kSfbOff % 8 == 0 &&
                   kSfCol + 2 * kSfBufCols <= kTmemCols,
               "TMEM budget");
 
-// tile rows of the block-scale layouts (activations: 128-row tiles of atoms; weights: 224-row
+// tile rows of the block-scale layouts (activations: 128-row tiles of atoms; weights: 192-row
 // tiles of images)
 constexpr int kSfTileA = BMC;
 constexpr int kSfTileB = BN;
@@ -79,7 +74,7 @@ constexpr int kEpiBufs = 1;
 constexpr int kEpiSmem = kEpiWarps * kEpiBufs * gemm_common::kStageBytes;
 
 constexpr int kTA = BMC * BKB;               // 16 KB
-constexpr int kTB = BNC * BKB;               // 14 KB
+constexpr int kTB = BNC * BKB;               // 12 KB
 // Scale chunks hold 4 scales per row and cover 64 K: 4 per stage.
 constexpr int kSfK = 64;
 constexpr int kSfChunks = BKB * 2 / kSfK;                // per stage
